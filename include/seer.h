@@ -1,0 +1,200 @@
+/*
+ * seer.h -- C ABI of the B200 (sm_100a) gated block-sparse decode library.
+ *
+ * The library computes one decode step of SeerAttention-R's sparse attention
+ * over a grouped-query (GQA) KV cache:
+ *
+ *   a1 seer_kpool_update   pooled-and-projected K per KV block (the gate's
+ *                          key side, kept as a cache)
+ *   a2 seer_gate_scores    one gating score per (batch, KV head, block) from
+ *                          the un-pooled decode query
+ *   a3 seer_select_blocks  the kept blocks under a token budget
+ *   a4 seer_sparse_decode  split-KV flash-decode over the kept blocks only
+ *   a5 seer_combine        merge of the split partials into the output
+ *
+ * Sources: "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
+ * (abstract) for the decode setting, the un-pooled query, the token budget and
+ * the 64/128 block sizes; "SeerAttention: Learning Intrinsic Sparse Attention
+ * in Your LLMs" (abstract) for the gate itself (pool along the sequence,
+ * learnable linear layers, multiply to get block scores).
+ *
+ * Conventions shared by every call:
+ *  - All tensor arguments are DEVICE pointers to dense row-major arrays with
+ *    the shapes given below. The caller allocates, owns and frees every
+ *    buffer; the library never allocates, frees or synchronises, and keeps no
+ *    state between calls.
+ *  - `dims` is read during the call only. NBmax = ceil(max_seq_len /
+ *    block_size) and G = num_q_heads / num_kv_heads.
+ *  - bf16 arrays are passed as `const void*` (IEEE bfloat16, 2 bytes).
+ *  - Work is enqueued on `stream` (NULL: the legacy default stream); calls
+ *    return before it runs.
+ *  - Arguments are validated on the host before anything is launched: a bad
+ *    pointer or shape returns SEER_ERR_INVALID_ARG, an unsupported size
+ *    SEER_ERR_UNSUPPORTED, and nothing is enqueued. A failed launch returns
+ *    SEER_ERR_CUDA. Faults inside a kernel surface at the caller's next
+ *    synchronisation, as for any CUDA kernel.
+ *  - Values held in device memory (sequence lengths, block lists) cannot be
+ *    checked on the host. A sequence length of 0 means an empty row (no block
+ *    kept, output 0, lse -inf); lengths above max_seq_len are clamped to it;
+ *    block indices outside [0, NB_b) are skipped by the decode kernel.
+ *  - Supported sizes: head_dim in {64, 128}, gate_dim in {64, 128},
+ *    block_size in {64, 128}, 1 <= G <= 8, num_q_heads % num_kv_heads == 0,
+ *    max_seq_len <= 2^24, batch * num_kv_heads * max_seq_len < 2^31.
+ */
+#ifndef SEER_H_
+#define SEER_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SEER_OK = 0,
+    SEER_ERR_INVALID_ARG = 1,
+    SEER_ERR_UNSUPPORTED = 2,
+    SEER_ERR_CUDA = 3
+} seer_status;
+
+typedef struct {
+    int32_t batch;        /* B */
+    int32_t num_q_heads;  /* Hq */
+    int32_t num_kv_heads; /* Hkv; G = Hq / Hkv query heads share one KV head */
+    int32_t head_dim;     /* D */
+    int32_t gate_dim;     /* dg, width of the gate's projected space */
+    int32_t block_size;   /* blk, tokens per sparse-attention block */
+    int32_t max_seq_len;  /* Lmax, tokens allocated per (b, kv head) in the caches */
+} seer_dims;
+
+/*
+ * a1. Pooled-K cache update ("SeerAttention", abstract: the gate pools K along
+ * the sequence dimension and passes it through a learnable linear layer).
+ *
+ * For every block j that holds a token in [upd_start[b], L_b), with
+ * L_b = seq_lens[b] and n_j the number of its tokens below L_b:
+ *     kpool[b,kvh,j,:] = W_k[kvh] . ( (1/n_j) * sum_{t in block j, t < L_b} K[b,kvh,t,:] )
+ * Other blocks are left untouched. upd_start = NULL rebuilds every block
+ * (after a prefill); upd_start[b] = L_b - 1 refreshes only the open last
+ * block (a decode step). Pooling and projection accumulate in fp32.
+ *
+ *   k_cache   bf16 [B, Hkv, Lmax, D]
+ *   w_k       fp32 [Hkv, dg, D]
+ *   seq_lens  int32 [B]
+ *   upd_start int32 [B] or NULL
+ *   kpool     fp32 [B, Hkv, NBmax, dg]   (output)
+ */
+seer_status seer_kpool_update(const seer_dims* dims, const void* k_cache, const float* w_k,
+                              const int32_t* seq_lens, const int32_t* upd_start, float* kpool,
+                              cudaStream_t stream);
+
+/*
+ * a2. Gate scores ("SeerAttention-R", abstract: query pooling removed for
+ * decoding, so the decode query is used as is; "SeerAttention", abstract: the
+ * projected query and key are multiplied to give block scores).
+ *
+ *     s[b,kvh,j] = (1/G) sum_{h in group(kvh)} (W_q[kvh] . q[b,h,:]) . kpool[b,kvh,j,:] / sqrt(dg)
+ * for j < NB_b = ceil(L_b / blk); entries j >= NB_b are not written.
+ *
+ *   q        bf16 [B, Hq, D]      (the decode query, one token per sequence)
+ *   w_q      fp32 [Hkv, dg, D]
+ *   kpool    fp32 [B, Hkv, NBmax, dg]
+ *   seq_lens int32 [B]
+ *   scores   fp32 [B, Hkv, NBmax]  (output)
+ */
+seer_status seer_gate_scores(const seer_dims* dims, const void* q, const float* w_q,
+                             const float* kpool, const int32_t* seq_lens, float* scores,
+                             cudaStream_t stream);
+
+/*
+ * a3. Block selection under a token budget ("SeerAttention-R", abstract: a
+ * 4K-token budget at block sizes 64/128).
+ *
+ * kmax = budget_tokens / block_size, k_b = min(kmax, NB_b). Row (b, kvh)
+ * keeps block NB_b - 1 (the open, possibly partial, last block) and the
+ * k_b - 1 highest-scoring blocks among 0 .. NB_b - 2; equal scores are
+ * broken toward the lower block index. The kept indices are written in
+ * ascending order to block_idx[b,kvh,0..k_b-1], the remaining slots get -1,
+ * and num_selected[b,kvh] = k_b.
+ *
+ *   scores        fp32 [B, Hkv, NBmax]
+ *   seq_lens      int32 [B]
+ *   budget_tokens a positive multiple of block_size
+ *   block_idx     int32 [B, Hkv, kmax]  (output)
+ *   num_selected  int32 [B, Hkv]        (output)
+ * Errors: budget_tokens not a positive multiple of block_size, or
+ * NBmax > 16384, give SEER_ERR_INVALID_ARG / SEER_ERR_UNSUPPORTED.
+ */
+seer_status seer_select_blocks(const seer_dims* dims, const float* scores, const int32_t* seq_lens,
+                               int32_t budget_tokens, int32_t* block_idx, int32_t* num_selected,
+                               cudaStream_t stream);
+
+/*
+ * a4. Block-sparse split-KV flash-decode ("SeerAttention-R", abstract: a
+ * sparse decoding kernel that reads only the kept blocks).
+ *
+ * For each query head h of KV head kvh, softmax attention of q[b,h] over the
+ * tokens t < L_b of the blocks listed in block_idx[b,kvh,0..num_selected-1]:
+ *     z_t = sm_scale * q[b,h,:] . K[b,kvh,t,:],   out = sum_t softmax(z)_t V[b,kvh,t,:]
+ * computed as partial results over disjoint pieces of the block list. Slot s
+ * of (b, h) receives the normalised partial output o_part[b,h,s,:] and its
+ * log-denominator lse_part[b,h,s] (natural log, scaled logits); a slot with
+ * no tokens has lse_part = -inf and its o_part is not written. seer_combine
+ * merges the slots.
+ *
+ * Scheduling: the kernel is persistent. The kept blocks of all rows, laid end
+ * to end with kmax positions reserved per row, are cut into P equal ranges,
+ * one per CTA; each (CTA, row) overlap is one slot. P is the device's SM
+ * count when num_splits >= min(kmax, SMs), else num_splits, so that no row
+ * ever needs more than num_splits slots. seer_default_num_splits() returns
+ * min(kmax, SMs).
+ *
+ *   q            bf16 [B, Hq, D]
+ *   k_cache      bf16 [B, Hkv, Lmax, D]
+ *   v_cache      bf16 [B, Hkv, Lmax, D]
+ *   seq_lens     int32 [B]
+ *   block_idx    int32 [B, Hkv, kmax]   (any order; a dense decode passes 0..NB_b-1)
+ *   num_selected int32 [B, Hkv]          (values above kmax are clamped to kmax)
+ *   kmax         row stride of block_idx, >= 1
+ *   num_splits   S, slots per (b, h), >= 1
+ *   sm_scale     softmax scale; <= 0 selects 1/sqrt(D)
+ *   o_part       fp32 [B, Hq, S, D]     (output)
+ *   lse_part     fp32 [B, Hq, S]        (output)
+ * The K/V caches must be 16-byte aligned (TMA); bf16 values only.
+ */
+seer_status seer_sparse_decode(const seer_dims* dims, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* seq_lens, const int32_t* block_idx,
+                               const int32_t* num_selected, int32_t kmax, int32_t num_splits,
+                               float sm_scale, float* o_part, float* lse_part, cudaStream_t stream);
+
+/*
+ * a5. Merge of the split partials (log-sum-exp weighted):
+ *     M = max_s lse_s,  w_s = exp(lse_s - M),
+ *     out = sum_s w_s o_s / sum_s w_s,  lse = M + log(sum_s w_s)
+ * Slots with lse = -inf are skipped; if every slot is -inf, out = 0 and
+ * lse = -inf.
+ *
+ *   o_part     fp32 [B, Hq, S, D]
+ *   lse_part   fp32 [B, Hq, S]
+ *   num_splits S, as passed to seer_sparse_decode
+ *   out        bf16 [B, Hq, D]   (output)
+ *   lse_out    fp32 [B, Hq]      (output, may be NULL)
+ */
+seer_status seer_combine(const seer_dims* dims, const float* o_part, const float* lse_part,
+                         int32_t num_splits, void* out, float* lse_out, cudaStream_t stream);
+
+/*
+ * Slots per (b, h) that let seer_sparse_decode use every SM of the current
+ * device: min(kmax, number of SMs). Host-only query (no launch).
+ */
+seer_status seer_default_num_splits(int32_t kmax, int32_t* num_splits);
+
+/* A short static description of a status code. */
+const char* seer_status_string(seer_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEER_H_ */
