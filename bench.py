@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of one gated block-sparse decode step on B200.
+
+A step is the whole hot path on one batch: kpool refresh of the open block,
+gate scores, block selection, split-KV sparse decode, combine. Inputs are
+seeded synthetic tensors resident in HBM before timing starts. Before every
+timed step a 256 MiB memset flushes L2 and a short device sleep lets the host
+enqueue the step ahead of the GPU; neither is inside the timed interval,
+which runs from an event before the first launch of the step to an event
+after the last (CUDA events on the launching stream). The sparse decode
+kernel alone is bracketed by its own pair of events inside each step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); the path has no exchange step, so
+each rank runs an independent replica batch (weak scaling) and the step time
+is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode attention µs/step and HBM GB/s vs ~8 TB/s at 90% sparsity"
+UNIT = "us/step"
+DEFAULT_WORKLOAD = "decode_b16"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sparse_decode_traffic.json")
+DECODE_SRC = os.path.join(ROOT, "block_sparse_attention_seer_b200", "csrc", "sparse_decode.cu")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--e2e-steps", type=int, default=200)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- shared helpers
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(wl, seq_lens, block_idx, num_selected):
+    """Bytes the step must move: kept K+V tokens, the pooled-K scan, q and out.
+
+    Returns (step_bytes, decode_kernel_bytes, kept_tokens, kept_blocks).
+    """
+    B, Hkv, D, dg, blk = wl.batch, wl.num_kv_heads, wl.head_dim, wl.gate_dim, wl.block_size
+    toks = 0
+    blocks = 0
+    nb_total = 0
+    for b in range(B):
+        L = int(seq_lens[b])
+        nb = -(-L // blk)
+        nb_total += nb * Hkv
+        for h in range(Hkv):
+            n = int(num_selected[b, h])
+            for j in block_idx[b, h, :n]:
+                j = int(j)
+                if 0 <= j < nb:
+                    toks += min(blk, L - j * blk)
+                    blocks += 1
+    kv = toks * D * 2 * 2
+    qo = 2 * B * wl.num_q_heads * D * 2
+    kp = nb_total * dg * 4
+    return kv + kp + qo, kv + qo // 2, toks, blocks
+
+
+def recorded_traffic(kernel_launch_bytes_scale=1.0):
+    """DRAM traffic per decode launch from the committed ncu summary, if the kernel is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        src = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
+        if d.get("source_sha256") != src:
+            return None
+        return d
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def smi_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+def oracle_sample_time(wl, host, target_s):
+    """Time the fp64 oracle step (as it stands) on the first n batch entries; scale to the whole batch.
+
+    Returns (us_per_full_step, threads, description).
+    """
+    from oracle import oracle as O
+    O.build()
+
+    def run(n):
+        q, k, v = host["q"][:n], host["k"][:n], host["v"][:n]
+        t0 = time.perf_counter()
+        O.step(q, k, v, host["w_q"], host["w_k"], host["lens"][:n], wl.block_size, wl.budget_tokens)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    n = max(1, min(wl.batch, int(target_s / max(t1, 1e-3))))
+    reps = 1
+    t = run(n) if n > 1 else t1
+    while t * (reps + 1) / reps < target_s and reps < 50 and t < target_s / 2:
+        t += run(n)
+        reps += 1
+    per_call = t / reps
+    us = per_call * wl.batch / n * 1e6
+    desc = (f"oracle step (pool all blocks, gate, select, attend; fp64) on the first {n} of {wl.batch} batch "
+            f"entries ({n * wl.num_kv_heads} of {wl.batch * wl.num_kv_heads} (b, kv-head) rows), {reps} run(s), "
+            f"scaled by {wl.batch}/{n}")
+    return us, O.num_threads(), desc
+
+
+def host_inputs(inp):
+    from block_sparse_attention_seer_b200 import workloads as W
+    return dict(q=W.bf16_bits(inp["q"]), k=W.bf16_bits(inp["k_cache"]), v=W.bf16_bits(inp["v_cache"]),
+                w_q=inp["w_q"].cpu().numpy(), w_k=inp["w_k"].cpu().numpy(),
+                lens=np.asarray(inp["seq_lens_host"], np.int32))
+
+
+# ---------------------------------------------------------------- reference arm: the oracle on host cores
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from block_sparse_attention_seer_b200 import workloads as W
+    from oracle import oracle as O
+    O.build()
+    wl = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(wl, seed=args.seed, device="cpu")
+    host = host_inputs(inp)
+    total_budget = 150.0
+    n_steps = args.steps + args.warmup
+    per_step = total_budget / max(1, n_steps)
+    # size the per-step sample (batch entries) to the per-step budget
+    t0 = time.perf_counter()
+    O.step(host["q"][:1], host["k"][:1], host["v"][:1], host["w_q"], host["w_k"], host["lens"][:1],
+           wl.block_size, wl.budget_tokens)
+    t1 = time.perf_counter() - t0
+    n = max(1, min(wl.batch, int(per_step / max(t1, 1e-4))))
+    times = []
+    for i in range(n_steps):
+        t0 = time.perf_counter()
+        O.step(host["q"][:n], host["k"][:n], host["v"][:n], host["w_q"], host["w_k"], host["lens"][:n],
+               wl.block_size, wl.budget_tokens)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    us = float(np.mean(times)) * wl.batch / n * 1e6
+    desc = (f"oracle step on the first {n} of {wl.batch} batch entries per step, scaled by {wl.batch}/{n}")
+    line = {"impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "description": wl.description},
+            "cpu_baseline": {"value": us, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle", "sample": desc},
+            "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    del torch
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_attention_seer_b200 import api
+    from block_sparse_attention_seer_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(wl, seed=args.seed + rank, device=dev)
+    st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
+    st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
+    st.set_update_start(inp["seq_lens"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def run_step():
+        api.seer_kpool_update(st.dims, inp["k_cache"], inp["w_k"], inp["seq_lens"], st.upd_start, st.kpool)
+        api.seer_gate_scores(st.dims, inp["q"], inp["w_q"], st.kpool, inp["seq_lens"], st.scores)
+        api.seer_select_blocks(st.dims, st.scores, inp["seq_lens"], st.budget_tokens, st.block_idx,
+                               st.num_selected)
+
+    o_part, lse_part = st.parts(st.num_splits)
+
+    def run_decode():
+        api.seer_sparse_decode(st.dims, inp["q"], inp["k_cache"], inp["v_cache"], inp["seq_lens"], st.block_idx,
+                               st.num_selected, st.kmax, st.num_splits, 0.0, o_part, lse_part)
+
+    def run_combine():
+        api.seer_combine(st.dims, o_part, lse_part, st.num_splits, st.out, st.lse)
+
+    def one(evs=None):
+        flush.zero_()
+        torch.cuda._sleep(300_000)  # ~0.15 ms at 2 GHz: the host enqueues the step ahead of the GPU
+        if evs:
+            evs[0].record(stream)
+        run_step()
+        if evs:
+            evs[1].record(stream)
+        run_decode()
+        if evs:
+            evs[2].record(stream)
+        run_combine()
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(smi_index(local))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        one(ev[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = np.array([e[0].elapsed_time(e[3]) for e in ev])
+    dec_ms = np.array([e[1].elapsed_time(e[2]) for e in ev])
+    gate_ms = np.array([e[0].elapsed_time(e[1]) for e in ev])
+    ms_step = float(step_ms.mean())
+    ms_dec = float(dec_ms.mean())
+    if world > 1:
+        t = torch.tensor([ms_step, ms_dec], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, ms_dec = float(t[0]), float(t[1])
+
+    lens = inp["seq_lens_host"]
+    bidx = st.block_idx.cpu().numpy()
+    nsel = st.num_selected.cpu().numpy()
+    step_bytes, dec_bytes, toks, blocks = algorithmic_bytes(wl, lens, bidx, nsel)
+    peak, peak_kind = measured_peak()
+    achieved = dec_bytes / (ms_dec * 1e-3) / 1e9
+    traffic = recorded_traffic()
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "kernel": "sparse_decode",
+                "traffic": (traffic["dram_bytes_per_launch"] if traffic else None),
+                "algorithmic_bytes_per_launch": dec_bytes}
+
+    # ---- end to end through the public API: host inputs in, host output out, every step
+    e2e = None
+    if args.e2e_steps > 0:
+        B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
+        q_h = inp["q"].cpu().pin_memory()
+        kn_h = inp["k_cache"][:, :, int(lens[0]) - 1, :].contiguous().cpu().pin_memory()
+        vn_h = inp["v_cache"][:, :, int(lens[0]) - 1, :].contiguous().cpu().pin_memory()
+        out_h = torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory()
+        uniform = bool((lens == lens[0]).all())
+        pos = int(lens[0]) - 1
+        h2d = q_h.numel() * 2 + (kn_h.numel() + vn_h.numel()) * 2
+        d2h = out_h.numel() * 2
+        e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
+        for k in range(args.e2e_steps + 5):
+            flush.zero_()
+            torch.cuda._sleep(300_000)
+            evs = e_ev[k - 5] if k >= 5 else None
+            if evs:
+                evs[0].record(stream)
+            inp["q"].copy_(q_h, non_blocking=True)
+            if uniform:
+                inp["k_cache"][:, :, pos, :].copy_(kn_h, non_blocking=True)
+                inp["v_cache"][:, :, pos, :].copy_(vn_h, non_blocking=True)
+            run_step()
+            run_decode()
+            run_combine()
+            out_h.copy_(st.out, non_blocking=True)
+            if evs:
+                evs[1].record(stream)
+        torch.cuda.synchronize()
+        e2e_us = float(np.mean([e[0].elapsed_time(e[1]) for e in e_ev])) * 1e3
+        if world > 1:
+            t = torch.tensor([e2e_us], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_us = float(t[0])
+        e2e = {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        us, cores, desc = oracle_sample_time(wl, host_inputs(inp), args.cpu_seconds)
+        cpu = {"value": round(us, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(ms_step * 1e3, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 KV cache and query, random N(0,1/D) gate weights)",
+            "config": {"workload": wl.name, "description": wl.description, "batch": wl.batch,
+                       "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                       "gate_dim": wl.gate_dim, "block_size": wl.block_size, "max_seq_len": wl.max_seq_len,
+                       "budget_tokens": wl.budget_tokens, "num_splits": st.num_splits,
+                       "kept_blocks": blocks, "kept_tokens": toks,
+                       "sparsity": round(1 - toks / float(sum(int(x) for x in lens) * wl.num_kv_heads), 4),
+                       "parallelism": f"replicas x{world}",
+                       "l2": "256 MiB memset before every step, outside the timed interval",
+                       "timing": "CUDA events per step on the launching stream; mean over steps; max over ranks"},
+            "step_bytes": step_bytes,
+            "step_hbm_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
+            "step_frac_of_8tbs": round(step_bytes / (ms_step * 1e-3) / 8e12, 4),
+            "decode_kernel_us": round(ms_dec * 1e3, 3),
+            "gate_select_us": round(float(gate_ms.mean()) * 1e3, 3),
+            "step_us_p50": round(float(np.median(step_ms)) * 1e3, 3),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 5 * args.steps,
+            "clocks": clocks,
+            "wall_s": round(wall, 3),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

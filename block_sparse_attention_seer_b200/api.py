@@ -1,0 +1,199 @@
+"""ctypes binding of ``libseer.so`` -- the names and arguments of include/seer.h.
+
+Argument marshalling only: tensors are passed as raw device pointers and the
+stream as its CUDA handle; every step of the computation runs in the CUDA
+library. Importing this module loads the library and raises if it has not
+been built -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "seer.h")
+
+SEER_OK, SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CUDA = 0, 1, 2, 3
+
+
+class SeerError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class seer_dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "num_q_heads", "num_kv_heads", "head_dim", "gate_dim", "block_size", "max_seq_len")]
+
+
+def _load_library():
+    path = _build.LIB
+    if not os.path.exists(path):
+        raise ImportError(f"libseer.so is not built ({path}); run "
+                          "`python -m block_sparse_attention_seer_b200.build` or __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    P, I32, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    D = ctypes.POINTER(seer_dims)
+    sig = {
+        "seer_kpool_update": [D, P, P, P, P, P, P],
+        "seer_gate_scores": [D, P, P, P, P, P, P],
+        "seer_select_blocks": [D, P, P, I32, P, P, P],
+        "seer_sparse_decode": [D, P, P, P, P, P, P, I32, I32, F32, P, P, P],
+        "seer_combine": [D, P, P, I32, P, P, P],
+        "seer_default_num_splits": [I32, P],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.seer_status_string.argtypes = [ctypes.c_int]
+    lib.seer_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+LIB = _load_library()
+
+
+def header_functions() -> list[str]:
+    """Entry points declared in include/seer.h."""
+    text = open(HEADER).read()
+    return re.findall(r"^\s*(?:seer_status|const char\*)\s+(seer_\w+)\s*\(", text, flags=re.M)
+
+
+def status_string(status: int) -> str:
+    return LIB.seer_status_string(int(status)).decode()
+
+
+def make_dims(batch, num_q_heads, num_kv_heads, head_dim, gate_dim, block_size, max_seq_len) -> seer_dims:
+    return seer_dims(batch, num_q_heads, num_kv_heads, head_dim, gate_dim, block_size, max_seq_len)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if not x.is_contiguous():
+            raise ValueError("tensor arguments must be contiguous")
+        return x.data_ptr()
+    raise TypeError(f"expected a tensor, int pointer or None, got {type(x)}")
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int):
+    if status != SEER_OK:
+        raise SeerError(fn, status)
+
+
+def seer_kpool_update(dims, k_cache, w_k, seq_lens, upd_start, kpool, stream=None):
+    _check("seer_kpool_update", LIB.seer_kpool_update(ctypes.byref(dims), _ptr(k_cache), _ptr(w_k), _ptr(seq_lens),
+                                                      _ptr(upd_start), _ptr(kpool), _stream(stream)))
+
+
+def seer_gate_scores(dims, q, w_q, kpool, seq_lens, scores, stream=None):
+    _check("seer_gate_scores", LIB.seer_gate_scores(ctypes.byref(dims), _ptr(q), _ptr(w_q), _ptr(kpool),
+                                                    _ptr(seq_lens), _ptr(scores), _stream(stream)))
+
+
+def seer_select_blocks(dims, scores, seq_lens, budget_tokens, block_idx, num_selected, stream=None):
+    _check("seer_select_blocks", LIB.seer_select_blocks(ctypes.byref(dims), _ptr(scores), _ptr(seq_lens),
+                                                        int(budget_tokens), _ptr(block_idx), _ptr(num_selected),
+                                                        _stream(stream)))
+
+
+def seer_sparse_decode(dims, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax, num_splits, sm_scale,
+                       o_part, lse_part, stream=None):
+    _check("seer_sparse_decode", LIB.seer_sparse_decode(
+        ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), _ptr(block_idx),
+        _ptr(num_selected), int(kmax), int(num_splits), float(sm_scale), _ptr(o_part), _ptr(lse_part),
+        _stream(stream)))
+
+
+def seer_combine(dims, o_part, lse_part, num_splits, out, lse_out, stream=None):
+    _check("seer_combine", LIB.seer_combine(ctypes.byref(dims), _ptr(o_part), _ptr(lse_part), int(num_splits),
+                                            _ptr(out), _ptr(lse_out), _stream(stream)))
+
+
+def seer_default_num_splits(kmax: int) -> int:
+    out = ctypes.c_int32(0)
+    _check("seer_default_num_splits", LIB.seer_default_num_splits(int(kmax), ctypes.byref(out)))
+    return int(out.value)
+
+
+class DecodeStep:
+    """Device buffers and the five calls of one decode step for fixed shapes.
+
+    Buffers are allocated once (torch owns them); each call only launches
+    kernels on the current stream. Launch count per ``step``: 5.
+    """
+
+    def __init__(self, batch, num_q_heads, num_kv_heads, head_dim, gate_dim, block_size, max_seq_len,
+                 budget_tokens, device="cuda", num_splits=None):
+        self.dims = make_dims(batch, num_q_heads, num_kv_heads, head_dim, gate_dim, block_size, max_seq_len)
+        self.budget_tokens = int(budget_tokens)
+        self.kmax = self.budget_tokens // block_size
+        nb_max = (max_seq_len + block_size - 1) // block_size
+        self.nb_max = nb_max
+        self.num_splits = int(num_splits) if num_splits else seer_default_num_splits(self.kmax)
+        dev = torch.device(device)
+        f32, i32 = torch.float32, torch.int32
+        self.kpool = torch.zeros(batch, num_kv_heads, nb_max, gate_dim, dtype=f32, device=dev)
+        self.scores = torch.zeros(batch, num_kv_heads, nb_max, dtype=f32, device=dev)
+        self.block_idx = torch.zeros(batch, num_kv_heads, self.kmax, dtype=i32, device=dev)
+        self.num_selected = torch.zeros(batch, num_kv_heads, dtype=i32, device=dev)
+        self.out = torch.zeros(batch, num_q_heads, head_dim, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.zeros(batch, num_q_heads, dtype=f32, device=dev)
+        self.upd_start = torch.zeros(batch, dtype=i32, device=dev)
+        self._parts = {}
+
+    def parts(self, num_splits):
+        if num_splits not in self._parts:
+            d = self.dims
+            dev = self.kpool.device
+            self._parts[num_splits] = (
+                torch.empty(d.batch, d.num_q_heads, num_splits, d.head_dim, dtype=torch.float32, device=dev),
+                torch.empty(d.batch, d.num_q_heads, num_splits, dtype=torch.float32, device=dev))
+        return self._parts[num_splits]
+
+    def build_pool(self, k_cache, w_k, seq_lens, stream=None):
+        """Pooled-K cache of every block (after a prefill)."""
+        seer_kpool_update(self.dims, k_cache, w_k, seq_lens, None, self.kpool, stream)
+
+    def set_update_start(self, seq_lens):
+        """Decode refresh point: the open last block (start = L_b - 1)."""
+        torch.sub(seq_lens, 1, out=self.upd_start)
+
+    def attend(self, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax, num_splits=None,
+               sm_scale=0.0, stream=None):
+        """a4 + a5 on a given block list (e.g. a dense list, or the oracle's)."""
+        S = int(num_splits) if num_splits else seer_default_num_splits(kmax)
+        o_part, lse_part = self.parts(S)
+        seer_sparse_decode(self.dims, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax, S, sm_scale,
+                           o_part, lse_part, stream)
+        seer_combine(self.dims, o_part, lse_part, S, self.out, self.lse, stream)
+        return self.out, self.lse
+
+    def step(self, q, k_cache, v_cache, w_q, w_k, seq_lens, sm_scale=0.0, stream=None):
+        """One decode step a1..a5; ``upd_start`` must hold the refresh points (set_update_start)."""
+        seer_kpool_update(self.dims, k_cache, w_k, seq_lens, self.upd_start, self.kpool, stream)
+        seer_gate_scores(self.dims, q, w_q, self.kpool, seq_lens, self.scores, stream)
+        seer_select_blocks(self.dims, self.scores, seq_lens, self.budget_tokens, self.block_idx, self.num_selected,
+                           stream)
+        return self.attend(q, k_cache, v_cache, seq_lens, self.block_idx, self.num_selected, self.kmax,
+                           self.num_splits, sm_scale, stream)
+
+    LAUNCHES_PER_STEP = 5

@@ -1,0 +1,158 @@
+// gate_scores.cu -- block gating scores from the un-pooled decode query.
+//
+// "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
+// (abstract) keeps SeerAttention's gate but removes query pooling, so the
+// single decode query is projected as is; "SeerAttention: Learning Intrinsic
+// Sparse Attention in Your LLMs" (abstract) multiplies the projected query
+// with the projected pooled keys to score each block. Per (b, kvh):
+//
+//   s[j] = (1/G) sum_h (W_q q_h) . kpool[j] / sqrt(dg)
+//        = (W_q qbar) . kpool[j] / sqrt(dg),   qbar = (1/G) sum_h q_h
+//
+// (the two forms agree by linearity; the second needs one projection). The
+// scan over kpool is the HBM cost. A thread-block cluster of C CTAs serves one
+// row: each CTA projects dg/C components of W_q qbar, the cluster exchanges
+// them through distributed shared memory, and each CTA then scores its own
+// contiguous chunk of the row's blocks, one warp per block row of kpool
+// (16-byte loads, shuffle reduction).
+#include <cooperative_groups.h>
+
+#include "seer_device.cuh"
+#include "seer_launch.h"
+
+namespace cg = cooperative_groups;
+
+namespace seer {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+template <int D, int DG>
+__global__ void __launch_bounds__(kThreads)
+    gate_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w_q,
+                       const float* __restrict__ kpool, const int32_t* __restrict__ seq_lens,
+                       float* __restrict__ scores, int Hq, int Hkv, int G, int blk, int Lmax, int NBmax) {
+    __shared__ float qbar[D];
+    __shared__ float qg_part[DG];  // components this CTA projects (others stay unused)
+    __shared__ float qg[DG];
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int csize = (int)cluster.num_blocks();
+    const int crank = (int)cluster.block_rank();
+    const int row = blockIdx.y;
+    const int b = row / Hkv, kvh = row - b * Hkv;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid < D) {
+        const __nv_bfloat16* qh = q + ((size_t)b * Hq + (size_t)kvh * G) * D + tid;
+        float s = 0.f;
+        for (int h = 0; h < G; ++h) s += __bfloat162float(qh[(size_t)h * D]);
+        qbar[tid] = s / (float)G;
+    }
+    __syncthreads();
+    constexpr int kVecD = D / 32;
+    {
+        float qv[kVecD];
+#pragma unroll
+        for (int u = 0; u < kVecD; ++u) qv[u] = qbar[lane * kVecD + u];
+        const int per = DG / csize;
+        const float* W = w_q + (size_t)kvh * DG * D;
+        for (int e = crank * per + warp; e < (crank + 1) * per; e += kWarps) {
+            const float* we = W + (size_t)e * D + lane * kVecD;
+            float d;
+            if constexpr (kVecD == 4) {
+                const float4 wv = *reinterpret_cast<const float4*>(we);
+                d = wv.x * qv[0] + wv.y * qv[1] + wv.z * qv[2] + wv.w * qv[3];
+            } else {
+                const float2 wv = *reinterpret_cast<const float2*>(we);
+                d = wv.x * qv[0] + wv.y * qv[1];
+            }
+            d = warp_sum(d);
+            if (lane == 0) qg_part[e] = d;
+        }
+    }
+    cluster.sync();
+    if (tid < DG) {
+        const int owner = tid / (DG / csize);
+        qg[tid] = *cluster.map_shared_rank(&qg_part[tid], owner);
+    }
+    cluster.sync();  // remote reads done before any CTA of the cluster moves on or exits
+
+    const int L = clamp_len(seq_lens[b], Lmax);
+    const int NB = (L + blk - 1) / blk;
+    const int per = (NB + csize - 1) / csize;
+    const int j0 = crank * per;
+    const int j1 = min(NB, j0 + per);
+    constexpr int kVecG = DG / 32;
+    float gv[kVecG];
+    const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
+#pragma unroll
+    for (int u = 0; u < kVecG; ++u) gv[u] = qg[lane * kVecG + u];
+    const float* kp = kpool + (size_t)row * NBmax * DG + lane * kVecG;
+    float* out = scores + (size_t)row * NBmax;
+    constexpr int kUnroll = 4;
+    for (int jb = j0 + warp * kUnroll; jb < j1; jb += kWarps * kUnroll) {
+        float d[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int j = jb + u;
+            d[u] = 0.f;
+            if (j < j1) {
+                const float* src = kp + (size_t)j * DG;
+                if constexpr (kVecG == 4) {
+                    const float4 v = __ldcs(reinterpret_cast<const float4*>(src));
+                    d[u] = v.x * gv[0] + v.y * gv[1] + v.z * gv[2] + v.w * gv[3];
+                } else {
+                    const float2 v = __ldcs(reinterpret_cast<const float2*>(src));
+                    d[u] = v.x * gv[0] + v.y * gv[1];
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) d[u] = warp_sum(d[u]);
+        if (lane < kUnroll && jb + lane < j1) {
+            float v = d[0];
+#pragma unroll
+            for (int u = 1; u < kUnroll; ++u) v = (lane == u) ? d[u] : v;
+            out[jb + lane] = v * inv_sqrt_dg;
+        }
+    }
+}
+
+template <int D, int DG>
+cudaError_t launch_impl(const Shape& s, const void* q, const float* w_q, const float* kpool,
+                        const int32_t* seq_lens, float* scores, int csize, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize, s.B * s.Hkv, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gate_scores_kernel<D, DG>, static_cast<const __nv_bfloat16*>(q), w_q, kpool,
+                              seq_lens, scores, s.Hq, s.Hkv, s.G, s.blk, s.Lmax, s.NBmax);
+}
+
+}  // namespace
+
+cudaError_t launch_gate_scores(const Shape& s, const void* q, const float* w_q, const float* kpool,
+                               const int32_t* seq_lens, float* scores, int num_sms, cudaStream_t stream) {
+    const int rows = s.B * s.Hkv;
+    int csize = 1;
+    while (csize < 8 && rows * csize < 2 * num_sms && s.NBmax / (2 * csize) >= 32) csize *= 2;
+    cudaError_t e;
+    if (s.D == 128 && s.dg == 128) e = launch_impl<128, 128>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
+    else if (s.D == 128 && s.dg == 64) e = launch_impl<128, 64>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
+    else if (s.D == 64 && s.dg == 128) e = launch_impl<64, 128>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
+    else e = launch_impl<64, 64>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace seer

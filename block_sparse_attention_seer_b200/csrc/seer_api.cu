@@ -1,0 +1,194 @@
+// seer_api.cu -- the extern "C" entry points declared in include/seer.h:
+// host-side validation, device-property lookup, TMA descriptor encoding, and
+// the kernel launches. No allocation, no synchronisation, no state kept
+// between calls beyond per-device constants (SM count) and the driver entry
+// point of the tensor-map encoder.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "seer.h"
+#include "seer_launch.h"
+
+namespace {
+
+using seer::Shape;
+
+constexpr int kMaxDevices = 64;
+int g_num_sms[kMaxDevices] = {0};
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return -1;
+    if (dev < kMaxDevices && g_num_sms[dev] > 0) return g_num_sms[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+    if (dev < kMaxDevices) g_num_sms[dev] = n;
+    return n;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Checks shared by every call; fills `s`.
+seer_status check_dims(const seer_dims* d, Shape& s) {
+    if (!d) return SEER_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 || d->max_seq_len < 1) return SEER_ERR_INVALID_ARG;
+    if (d->num_q_heads % d->num_kv_heads != 0) return SEER_ERR_INVALID_ARG;
+    const int G = d->num_q_heads / d->num_kv_heads;
+    if (G > 8) return SEER_ERR_UNSUPPORTED;
+    if (d->head_dim != 64 && d->head_dim != 128) return SEER_ERR_UNSUPPORTED;
+    if (d->gate_dim != 64 && d->gate_dim != 128) return SEER_ERR_UNSUPPORTED;
+    if (d->block_size != 64 && d->block_size != 128) return SEER_ERR_UNSUPPORTED;
+    if (d->max_seq_len > (1 << 24)) return SEER_ERR_UNSUPPORTED;
+    const long long rows = (long long)d->batch * d->num_kv_heads;
+    if (rows > 65535) return SEER_ERR_UNSUPPORTED;
+    if (rows * d->max_seq_len >= (1LL << 31)) return SEER_ERR_UNSUPPORTED;
+    if ((long long)d->batch * d->num_q_heads >= (1LL << 31) / 128) return SEER_ERR_UNSUPPORTED;
+    s.B = d->batch;
+    s.Hq = d->num_q_heads;
+    s.Hkv = d->num_kv_heads;
+    s.G = G;
+    s.D = d->head_dim;
+    s.dg = d->gate_dim;
+    s.blk = d->block_size;
+    s.Lmax = d->max_seq_len;
+    s.NBmax = (d->max_seq_len + d->block_size - 1) / d->block_size;
+    return SEER_OK;
+}
+
+seer_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SEER_OK : SEER_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D view [B*Hkv*Lmax rows, D cols] of a bf16 cache; box = 64 cols (128 B) x blk rows, 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)s.D, (cuuint64_t)s.B * s.Hkv * s.Lmax};
+    const cuuint64_t strides[1] = {(cuuint64_t)s.D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)s.blk};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+seer_status seer_kpool_update(const seer_dims* dims, const void* k_cache, const float* w_k,
+                              const int32_t* seq_lens, const int32_t* upd_start, float* kpool,
+                              cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!k_cache || !w_k || !seq_lens || !kpool) return SEER_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(w_k, 16)) return SEER_ERR_INVALID_ARG;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    return from_cuda(seer::launch_kpool_update(s, k_cache, w_k, seq_lens, upd_start, kpool, nsm, stream));
+}
+
+seer_status seer_gate_scores(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
+                             const int32_t* seq_lens, float* scores, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !w_q || !kpool || !seq_lens || !scores) return SEER_ERR_INVALID_ARG;
+    if (!aligned(w_q, 16) || !aligned(kpool, 16)) return SEER_ERR_INVALID_ARG;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    return from_cuda(seer::launch_gate_scores(s, q, w_q, kpool, seq_lens, scores, nsm, stream));
+}
+
+seer_status seer_select_blocks(const seer_dims* dims, const float* scores, const int32_t* seq_lens,
+                               int32_t budget_tokens, int32_t* block_idx, int32_t* num_selected,
+                               cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!scores || !seq_lens || !block_idx || !num_selected) return SEER_ERR_INVALID_ARG;
+    if (budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
+    if (s.NBmax > 16384) return SEER_ERR_UNSUPPORTED;
+    return from_cuda(
+        seer::launch_select_blocks(s, scores, seq_lens, budget_tokens / s.blk, block_idx, num_selected, stream));
+}
+
+seer_status seer_sparse_decode(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* seq_lens, const int32_t* block_idx, const int32_t* num_selected,
+                               int32_t kmax, int32_t num_splits, float sm_scale, float* o_part, float* lse_part,
+                               cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !k_cache || !v_cache || !seq_lens || !block_idx || !num_selected || !o_part || !lse_part)
+        return SEER_ERR_INVALID_ARG;
+    if (kmax < 1 || num_splits < 1) return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16)) return SEER_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
+    if ((long long)s.B * s.Hq * num_splits * s.D >= (1LL << 40)) return SEER_ERR_UNSUPPORTED;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, k_cache, s) || !encode_cache_map(&tmv, v_cache, s)) return SEER_ERR_CUDA;
+    seer::DecodeLaunch a;
+    a.q = q;
+    a.seq_lens = seq_lens;
+    a.block_idx = block_idx;
+    a.num_selected = num_selected;
+    a.o_part = o_part;
+    a.lse_part = lse_part;
+    a.kmax = kmax;
+    a.num_splits = num_splits;
+    a.sm_scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
+    return from_cuda(seer::launch_sparse_decode(s, a, tmk, tmv, nsm, stream));
+}
+
+seer_status seer_combine(const seer_dims* dims, const float* o_part, const float* lse_part, int32_t num_splits,
+                         void* out, float* lse_out, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!o_part || !lse_part || !out || num_splits < 1) return SEER_ERR_INVALID_ARG;
+    if (!aligned(o_part, 16) || !aligned(out, 8)) return SEER_ERR_INVALID_ARG;
+    return from_cuda(seer::launch_combine(s, o_part, lse_part, num_splits, out, lse_out, stream));
+}
+
+seer_status seer_default_num_splits(int32_t kmax, int32_t* num_splits) {
+    if (kmax < 1 || !num_splits) return SEER_ERR_INVALID_ARG;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    *num_splits = kmax < nsm ? kmax : nsm;
+    return SEER_OK;
+}
+
+const char* seer_status_string(seer_status status) {
+    switch (status) {
+        case SEER_OK: return "ok";
+        case SEER_ERR_INVALID_ARG: return "invalid argument";
+        case SEER_ERR_UNSUPPORTED: return "unsupported size";
+        case SEER_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

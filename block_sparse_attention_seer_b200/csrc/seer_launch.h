@@ -1,0 +1,47 @@
+// seer_launch.h -- host-side launchers of the kernels behind the C ABI.
+// Arguments are assumed validated by the caller (seer_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace seer {
+
+struct Shape {
+    int B, Hq, Hkv, G, D, dg, blk, Lmax, NBmax;
+};
+
+cudaError_t launch_kpool_update(const Shape& s, const void* k_cache, const float* w_k, const int32_t* seq_lens,
+                                const int32_t* upd_start, float* kpool, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_gate_scores(const Shape& s, const void* q, const float* w_q, const float* kpool,
+                               const int32_t* seq_lens, float* scores, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_select_blocks(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax,
+                                 int32_t* block_idx, int32_t* num_selected, cudaStream_t stream);
+
+struct DecodeLaunch {
+    const void* q;
+    const int32_t* seq_lens;
+    const int32_t* block_idx;
+    const int32_t* num_selected;
+    float* o_part;
+    float* lse_part;
+    int kmax;
+    int num_splits;
+    float sm_scale;
+};
+
+// tmap_k / tmap_v: 2-D bf16 maps over [B*Hkv*Lmax rows, D cols], box 64 x blk,
+// 128-byte swizzle (built by the caller).
+cudaError_t launch_sparse_decode(const Shape& s, const DecodeLaunch& a, const CUtensorMap& tmap_k,
+                                 const CUtensorMap& tmap_v, int num_sms, cudaStream_t stream);
+
+// Number of CTAs the decode kernel runs for these arguments (1 per SM at most).
+int sparse_decode_ctas(const Shape& s, int kmax, int num_splits, int num_sms);
+
+cudaError_t launch_combine(const Shape& s, const float* o_part, const float* lse_part, int num_splits,
+                           void* out, float* lse_out, cudaStream_t stream);
+
+}  // namespace seer

@@ -34,3 +34,12 @@ def oracle():
     from oracle import oracle as o
     o.build()
     return o
+
+
+def pytest_sessionstart(session):
+    # Build the CUDA library (nvcc cross-compiles without a GPU) and the oracle
+    # before collection, so host tests can load and inspect them.
+    from block_sparse_attention_seer_b200 import build as b
+    b.build()
+    from oracle import oracle as o
+    o.build()

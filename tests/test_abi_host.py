@@ -1,0 +1,90 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load, export every entry point include/seer.h declares, and
+reject bad arguments on the host with the documented status before touching
+the device.
+"""
+import ctypes
+import subprocess
+
+import pytest
+
+from block_sparse_attention_seer_b200 import api
+
+
+def test_header_declares_the_path_calls():
+    names = api.header_functions()
+    for n in ("seer_kpool_update", "seer_gate_scores", "seer_select_blocks", "seer_sparse_decode",
+              "seer_combine", "seer_status_string", "seer_default_num_splits"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", api._build.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in api.header_functions():
+        assert n in exported, n
+        assert hasattr(api.LIB, n)
+
+
+def test_status_strings():
+    assert api.status_string(0) == "ok"
+    assert api.status_string(1) == "invalid argument"
+    assert api.status_string(2) == "unsupported size"
+    assert api.status_string(3) == "CUDA error"
+
+
+def _dims(**kw):
+    d = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, gate_dim=128, block_size=64, max_seq_len=1024)
+    d.update(kw)
+    return api.make_dims(**d)
+
+
+FAKE = 1 << 20  # never dereferenced: validation fails before any launch
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(head_dim=96), api.SEER_ERR_UNSUPPORTED),
+    (dict(gate_dim=32), api.SEER_ERR_UNSUPPORTED),
+    (dict(block_size=32), api.SEER_ERR_UNSUPPORTED),
+    (dict(num_q_heads=18, num_kv_heads=2), api.SEER_ERR_UNSUPPORTED),   # G = 9
+    (dict(num_q_heads=7), api.SEER_ERR_INVALID_ARG),                     # not a multiple of Hkv
+    (dict(batch=0), api.SEER_ERR_INVALID_ARG),
+    (dict(max_seq_len=0), api.SEER_ERR_INVALID_ARG),
+    (dict(max_seq_len=(1 << 24) + 1), api.SEER_ERR_UNSUPPORTED),
+])
+def test_bad_dims_rejected(bad, status):
+    d = _dims(**bad)
+    st = api.LIB.seer_combine(ctypes.byref(d), FAKE, FAKE, 4, FAKE, None, None)
+    assert st == status
+    st = api.LIB.seer_sparse_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE, None)
+    assert st == status
+
+
+def test_null_pointers_and_bad_scalars_rejected():
+    d = _dims()
+    L = api.LIB
+    assert L.seer_kpool_update(None, FAKE, FAKE, FAKE, None, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_kpool_update(ctypes.byref(d), None, FAKE, FAKE, None, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_gate_scores(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, None, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_select_blocks(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_select_blocks(ctypes.byref(d), FAKE, FAKE, 0, FAKE, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_select_blocks(ctypes.byref(d), FAKE, FAKE, 64, None, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_sparse_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 0.0, FAKE, FAKE,
+                                None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_sparse_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 0, 0.0, FAKE, FAKE,
+                                None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_sparse_decode(ctypes.byref(d), FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 4, 0.0, FAKE, FAKE,
+                                None) == api.SEER_ERR_INVALID_ARG            # q not 16-byte aligned
+    assert L.seer_sparse_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 8, 4, float("nan"), FAKE,
+                                FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_combine(ctypes.byref(d), FAKE, FAKE, 0, FAKE, None, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_combine(ctypes.byref(d), None, FAKE, 4, FAKE, None, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_default_num_splits(0, ctypes.byref(ctypes.c_int32())) == api.SEER_ERR_INVALID_ARG
+
+
+def test_python_wrapper_raises_on_error():
+    with pytest.raises(api.SeerError) as e:
+        api.seer_combine(_dims(head_dim=96), FAKE, FAKE, 4, FAKE, None, stream=0)
+    assert e.value.status == api.SEER_ERR_UNSUPPORTED
