@@ -2,13 +2,15 @@
 """Benchmark of one gated block-sparse decode step on B200.
 
 A step is the whole hot path on one batch: kpool refresh of the open block,
-gate scores, block selection, split-KV sparse decode, combine. Inputs are
+gate scores, block selection, split-KV sparse decode and the merge of the
+split partials -- run as ONE cooperative launch (seer_decode_step). Inputs are
 seeded synthetic tensors resident in HBM before timing starts. Before every
 timed step a 256 MiB memset flushes L2 and a short device sleep lets the host
-enqueue the step ahead of the GPU; neither is inside the timed interval,
-which runs from an event before the first launch of the step to an event
-after the last (CUDA events on the launching stream). The sparse decode
-kernel alone is bracketed by its own pair of events inside each step.
+enqueue the step ahead of the GPU; neither is inside the timed interval, a
+pair of CUDA events on the launching stream around the step's launch.
+
+The same step as the five separate C calls is timed afterwards (secondary
+numbers, with the sparse decode kernel bracketed alone).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -50,6 +52,7 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--batch", type=int, default=0, help="override the workload's batch (small profiling cases)")
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -162,6 +165,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (every rank calls it, same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
 def smi_index(local_rank):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -218,6 +230,8 @@ def run_reference(args):
     from oracle import oracle as O
     O.build()
     wl = W.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
     inp = W.make_inputs(wl, seed=args.seed, device="cpu")
     host = host_inputs(inp)
     total_budget = 150.0
@@ -269,6 +283,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     wl = W.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
     inp = W.make_inputs(wl, seed=args.seed + rank, device=dev)
     st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
     st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
@@ -276,7 +292,10 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def run_step():
+    def run_fused():
+        st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+
+    def run_gate_calls():
         api.seer_kpool_update(st.dims, inp["k_cache"], inp["w_k"], inp["seq_lens"], st.upd_start, st.kpool)
         api.seer_gate_scores(st.dims, inp["q"], inp["w_q"], st.kpool, inp["seq_lens"], st.scores)
         api.seer_select_blocks(st.dims, st.scores, inp["seq_lens"], st.budget_tokens, st.block_idx,
@@ -291,12 +310,23 @@ def run_ours(args):
     def run_combine():
         api.seer_combine(st.dims, o_part, lse_part, st.num_splits, st.out, st.lse)
 
-    def one(evs=None):
+    def prepare():
         flush.zero_()
-        torch.cuda._sleep(300_000)  # ~0.15 ms at 2 GHz: the host enqueues the step ahead of the GPU
+        torch.cuda._sleep(300_000)  # ~0.15 ms: the host enqueues the step ahead of the GPU
+
+    def fused_once(evs=None):
+        prepare()
         if evs:
             evs[0].record(stream)
-        run_step()
+        run_fused()
+        if evs:
+            evs[1].record(stream)
+
+    def separate_once(evs=None):
+        prepare()
+        if evs:
+            evs[0].record(stream)
+        run_gate_calls()
         if evs:
             evs[1].record(stream)
         run_decode()
@@ -306,10 +336,12 @@ def run_ours(args):
         if evs:
             evs[3].record(stream)
 
+    st.set_update_start(inp["seq_lens"])
     for _ in range(args.warmup):
-        one()
+        fused_once()
+        separate_once()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(smi_index(local))
     sampler.start()
     time.sleep(0.3)
@@ -318,33 +350,45 @@ def run_ours(args):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for k in range(args.steps):
-        one(ev[k])
+        fused_once(ev[k])
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    step_ms = np.array([e[0].elapsed_time(e[3]) for e in ev])
-    dec_ms = np.array([e[1].elapsed_time(e[2]) for e in ev])
-    gate_ms = np.array([e[0].elapsed_time(e[1]) for e in ev])
+    step_ms = np.array([e[0].elapsed_time(e[1]) for e in ev])
     ms_step = float(step_ms.mean())
-    ms_dec = float(dec_ms.mean())
+
+    # the same step as five separate calls (secondary: per-kernel brackets)
+    n_sep = min(args.steps, 300)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_sep)]
+    for k in range(n_sep):
+        separate_once(sev[k])
+    torch.cuda.synchronize()
+    sep_step_ms = float(np.mean([e[0].elapsed_time(e[3]) for e in sev]))
+    ms_dec = float(np.mean([e[1].elapsed_time(e[2]) for e in sev]))
+    gate_ms = np.array([e[0].elapsed_time(e[1]) for e in sev])
     if world > 1:
-        t = torch.tensor([ms_step, ms_dec], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, ms_dec = float(t[0]), float(t[1])
+        ms_step, ms_dec, sep_step_ms = max_over_ranks([ms_step, ms_dec, sep_step_ms], dev)
 
     lens = inp["seq_lens_host"]
     bidx = st.block_idx.cpu().numpy()
     nsel = st.num_selected.cpu().numpy()
     step_bytes, dec_bytes, toks, blocks = algorithmic_bytes(wl, lens, bidx, nsel)
     peak, peak_kind = measured_peak()
-    achieved = dec_bytes / (ms_dec * 1e-3) / 1e9
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
     traffic = recorded_traffic()
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "kernel": "sparse_decode",
+                "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "kernel": "decode_step_kernel",
                 "traffic": (traffic["dram_bytes_per_launch"] if traffic else None),
-                "algorithmic_bytes_per_launch": dec_bytes}
+                "algorithmic_bytes_per_launch": step_bytes}
+    dec_achieved = dec_bytes / (ms_dec * 1e-3) / 1e9
+    separate = {"step_us": round(sep_step_ms * 1e3, 3), "launches_per_step": 5,
+                "gate_select_us": round(float(gate_ms.mean()) * 1e3, 3),
+                "sparse_decode_us": round(ms_dec * 1e3, 3),
+                "sparse_decode_bytes": dec_bytes,
+                "sparse_decode_gbs": round(dec_achieved, 1),
+                "sparse_decode_frac": round(dec_achieved / peak, 4)}
 
     # ---- end to end through the public API: host inputs in, host output out, every step
     e2e = None
@@ -369,18 +413,14 @@ def run_ours(args):
             if uniform:
                 inp["k_cache"][:, :, pos, :].copy_(kn_h, non_blocking=True)
                 inp["v_cache"][:, :, pos, :].copy_(vn_h, non_blocking=True)
-            run_step()
-            run_decode()
-            run_combine()
+            run_fused()
             out_h.copy_(st.out, non_blocking=True)
             if evs:
                 evs[1].record(stream)
         torch.cuda.synchronize()
         e2e_us = float(np.mean([e[0].elapsed_time(e[1]) for e in e_ev])) * 1e3
         if world > 1:
-            t = torch.tensor([e2e_us], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_us = float(t[0])
+            (e2e_us,) = max_over_ranks([e2e_us], dev)
         e2e = {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
@@ -407,13 +447,12 @@ def run_ours(args):
             "step_bytes": step_bytes,
             "step_hbm_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
             "step_frac_of_8tbs": round(step_bytes / (ms_step * 1e-3) / 8e12, 4),
-            "decode_kernel_us": round(ms_dec * 1e3, 3),
-            "gate_select_us": round(float(gate_ms.mean()) * 1e3, 3),
             "step_us_p50": round(float(np.median(step_ms)) * 1e3, 3),
+            "separate_calls": separate,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": args.steps,
             "clocks": clocks,
             "wall_s": round(wall, 3),
         }

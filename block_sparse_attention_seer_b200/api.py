@@ -23,7 +23,8 @@ SEER_OK, SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CUDA = 0, 1, 2, 3
 
 class SeerError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+        detail = f" [{LIB.seer_last_error_string().decode()}]" if status == SEER_ERR_CUDA else ""
+        super().__init__(f"{fn} failed: {status_string(status)} (status {status}){detail}")
         self.status = status
 
 
@@ -47,6 +48,10 @@ def _load_library():
         "seer_sparse_decode": [D, P, P, P, P, P, P, I32, I32, F32, P, P, P],
         "seer_combine": [D, P, P, I32, P, P, P],
         "seer_default_num_splits": [I32, P],
+        "seer_decode_wait_failures": [P, I32],
+        "seer_decode_step_workspace_size": [D, I32, P],
+        "seer_decode_step": [D, P, P, P, P, P, P, P, I32, F32, P, P, P, P, P, P, ctypes.c_size_t, P],
+        "seer_wait_selftest": [ctypes.c_int64, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -54,6 +59,8 @@ def _load_library():
         f.restype = ctypes.c_int
     lib.seer_status_string.argtypes = [ctypes.c_int]
     lib.seer_status_string.restype = ctypes.c_char_p
+    lib.seer_last_error_string.argtypes = []
+    lib.seer_last_error_string.restype = ctypes.c_char_p
     return lib
 
 
@@ -128,9 +135,37 @@ def seer_combine(dims, o_part, lse_part, num_splits, out, lse_out, stream=None):
                                             _ptr(out), _ptr(lse_out), _stream(stream)))
 
 
+def seer_decode_step_workspace_size(dims, budget_tokens) -> int:
+    out = ctypes.c_size_t(0)
+    _check("seer_decode_step_workspace_size",
+           LIB.seer_decode_step_workspace_size(ctypes.byref(dims), int(budget_tokens), ctypes.byref(out)))
+    return int(out.value)
+
+
+def seer_decode_step(dims, q, k_cache, v_cache, w_q, w_k, seq_lens, upd_start, budget_tokens, sm_scale, kpool,
+                     block_idx, num_selected, out, lse_out, workspace, workspace_bytes=None, stream=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else int(workspace_bytes)
+    _check("seer_decode_step", LIB.seer_decode_step(
+        ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(w_q), _ptr(w_k), _ptr(seq_lens),
+        _ptr(upd_start), int(budget_tokens), float(sm_scale), _ptr(kpool), _ptr(block_idx), _ptr(num_selected),
+        _ptr(out), _ptr(lse_out), _ptr(workspace), nbytes, _stream(stream)))
+
+
 def seer_default_num_splits(kmax: int) -> int:
     out = ctypes.c_int32(0)
     _check("seer_default_num_splits", LIB.seer_default_num_splits(int(kmax), ctypes.byref(out)))
+    return int(out.value)
+
+
+def seer_decode_wait_failures(reset: bool = False) -> int:
+    out = ctypes.c_uint32(0)
+    _check("seer_decode_wait_failures", LIB.seer_decode_wait_failures(ctypes.byref(out), int(bool(reset))))
+    return int(out.value)
+
+
+def seer_wait_selftest(limit_ns: int) -> int:
+    out = ctypes.c_int32(-1)
+    _check("seer_wait_selftest", LIB.seer_wait_selftest(int(limit_ns), ctypes.byref(out)))
     return int(out.value)
 
 
@@ -185,6 +220,20 @@ class DecodeStep:
         seer_sparse_decode(self.dims, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax, S, sm_scale,
                            o_part, lse_part, stream)
         seer_combine(self.dims, o_part, lse_part, S, self.out, self.lse, stream)
+        return self.out, self.lse
+
+    def workspace(self):
+        """Zero-filled scratch of the fused step (allocated once; each call leaves it ready for the next)."""
+        if getattr(self, "_ws", None) is None:
+            n = seer_decode_step_workspace_size(self.dims, self.budget_tokens)
+            self._ws = torch.zeros(n, dtype=torch.uint8, device=self.kpool.device)
+        return self._ws
+
+    def fused_step(self, q, k_cache, v_cache, w_q, w_k, seq_lens, sm_scale=0.0, stream=None, upd_start=None):
+        """One decode step a1..a5 in a single cooperative launch (seer_decode_step)."""
+        seer_decode_step(self.dims, q, k_cache, v_cache, w_q, w_k, seq_lens, upd_start, self.budget_tokens,
+                         sm_scale, self.kpool, self.block_idx, self.num_selected, self.out, self.lse,
+                         self.workspace(), stream=stream)
         return self.out, self.lse
 
     def step(self, q, k_cache, v_cache, w_q, w_k, seq_lens, sm_scale=0.0, stream=None):

@@ -17,7 +17,7 @@
 // (16-byte loads, shuffle reduction).
 #include <cooperative_groups.h>
 
-#include "seer_device.cuh"
+#include "gate_core.cuh"
 #include "seer_launch.h"
 
 namespace cg = cooperative_groups;
@@ -44,12 +44,7 @@ __global__ void __launch_bounds__(kThreads)
     const int b = row / Hkv, kvh = row - b * Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    if (tid < D) {
-        const __nv_bfloat16* qh = q + ((size_t)b * Hq + (size_t)kvh * G) * D + tid;
-        float s = 0.f;
-        for (int h = 0; h < G; ++h) s += __bfloat162float(qh[(size_t)h * D]);
-        qbar[tid] = s / (float)G;
-    }
+    group_query_mean<D>(q + ((size_t)b * Hq + (size_t)kvh * G) * D, G, qbar);
     __syncthreads();
     constexpr int kVecD = D / 32;
     {
@@ -57,20 +52,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int u = 0; u < kVecD; ++u) qv[u] = qbar[lane * kVecD + u];
         const int per = DG / csize;
-        const float* W = w_q + (size_t)kvh * DG * D;
-        for (int e = crank * per + warp; e < (crank + 1) * per; e += kWarps) {
-            const float* we = W + (size_t)e * D + lane * kVecD;
-            float d;
-            if constexpr (kVecD == 4) {
-                const float4 wv = *reinterpret_cast<const float4*>(we);
-                d = wv.x * qv[0] + wv.y * qv[1] + wv.z * qv[2] + wv.w * qv[3];
-            } else {
-                const float2 wv = *reinterpret_cast<const float2*>(we);
-                d = wv.x * qv[0] + wv.y * qv[1];
-            }
-            d = warp_sum(d);
-            if (lane == 0) qg_part[e] = d;
-        }
+        warp_matvec_rows<D>(w_q + (size_t)kvh * DG * D, qv, crank * per + warp, (crank + 1) * per, kWarps,
+                            [&](int e, float x) { qg_part[e] = x; });
     }
     cluster.sync();
     if (tid < DG) {
@@ -89,33 +72,25 @@ __global__ void __launch_bounds__(kThreads)
     const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
 #pragma unroll
     for (int u = 0; u < kVecG; ++u) gv[u] = qg[lane * kVecG + u];
-    const float* kp = kpool + (size_t)row * NBmax * DG + lane * kVecG;
+    using Vec = GateVec<DG>;
+    const Vec* kp = reinterpret_cast<const Vec*>(kpool + (size_t)row * NBmax * DG) + lane;
     float* out = scores + (size_t)row * NBmax;
-    constexpr int kUnroll = 4;
+    constexpr int kUnroll = 8;
     for (int jb = j0 + warp * kUnroll; jb < j1; jb += kWarps * kUnroll) {
-        float d[kUnroll];
+        Vec v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int j = jb + u;
-            d[u] = 0.f;
-            if (j < j1) {
-                const float* src = kp + (size_t)j * DG;
-                if constexpr (kVecG == 4) {
-                    const float4 v = __ldcs(reinterpret_cast<const float4*>(src));
-                    d[u] = v.x * gv[0] + v.y * gv[1] + v.z * gv[2] + v.w * gv[3];
-                } else {
-                    const float2 v = __ldcs(reinterpret_cast<const float2*>(src));
-                    d[u] = v.x * gv[0] + v.y * gv[1];
-                }
-            }
+            const int j = min(jb + u, j1 - 1);  // clamped duplicate loads past j1 are never stored
+            v[u] = __ldcs(kp + (size_t)j * (DG / kVecG));
         }
+        float d[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) d[u] = warp_sum(d[u]);
+        for (int u = 0; u < kUnroll; ++u) d[u] = gate_dot<DG>(v[u], gv);
         if (lane < kUnroll && jb + lane < j1) {
-            float v = d[0];
+            float x = d[0];
 #pragma unroll
-            for (int u = 1; u < kUnroll; ++u) v = (lane == u) ? d[u] : v;
-            out[jb + lane] = v * inv_sqrt_dg;
+            for (int u = 1; u < kUnroll; ++u) x = (lane == u) ? d[u] : x;
+            out[jb + lane] = x * inv_sqrt_dg;
         }
     }
 }
@@ -151,7 +126,10 @@ cudaError_t launch_gate_scores(const Shape& s, const void* q, const float* w_q, 
     else if (s.D == 128 && s.dg == 64) e = launch_impl<128, 64>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
     else if (s.D == 64 && s.dg == 128) e = launch_impl<64, 128>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
     else e = launch_impl<64, 64>(s, q, w_q, kpool, seq_lens, scores, csize, stream);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // a rejected launch must not leak into the next call
+        return e;
+    }
     return cudaGetLastError();
 }
 

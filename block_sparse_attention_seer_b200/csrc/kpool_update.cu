@@ -7,10 +7,11 @@
 //   kpool[b,kvh,j,:] = W_k[kvh] . mean_{t in block j, t < L_b} K[b,kvh,t,:]
 //
 // One CTA (128 threads) per (row, chunk); it walks blocks j = j_first + chunk,
-// + chunks, ... below NB_b. The pool reads each block's tokens with 16-byte
-// vector loads and accumulates in fp32 in a fixed order; the projection is a
-// warp-per-output-row dot product against W_k (read from L2).
-#include "seer_device.cuh"
+// + chunks, ... below NB_b. The pool (gate_core.cuh) loads all of a thread's
+// token rows with 16-byte vector loads before summing them in fp32 in a fixed
+// order; the projection is one warp per output row against W_k, eight rows
+// in flight per warp.
+#include "gate_core.cuh"
 #include "seer_launch.h"
 
 namespace seer {
@@ -18,70 +19,31 @@ namespace {
 
 constexpr int kThreads = 128;
 
-template <int D>
+template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads)
     kpool_update_kernel(const __nv_bfloat16* __restrict__ k_cache, const float* __restrict__ w_k,
                         const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ upd_start,
-                        float* __restrict__ kpool, int Hkv, int Lmax, int blk, int dg, int NBmax, int chunks) {
-    constexpr int kLanesPerRow = D / 8;                 // 16-byte pieces per token row
-    constexpr int kRowsPerPass = kThreads / kLanesPerRow;
-    __shared__ float red[kRowsPerPass][D];
-    __shared__ float pooled[D];
-
+                        float* __restrict__ kpool, int Hkv, int Lmax, int dg, int NBmax, int chunks) {
+    __shared__ PoolSmem<D> sm;
     const int row = blockIdx.y;
     const int b = row / Hkv, kvh = row - b * Hkv;
     const int L = clamp_len(seq_lens[b], Lmax);
-    const int NB = (L + blk - 1) / blk;
+    const int NB = (L + BLK - 1) / BLK;
     int start = upd_start ? upd_start[b] : 0;
     start = start < 0 ? 0 : start;
-    const int j_first = start / blk;
-    const int tid = threadIdx.x;
-    const int rsub = tid / kLanesPerRow, cpart = tid % kLanesPerRow;
-    const int warp = tid >> 5, lane = tid & 31;
+    const int j_first = start / BLK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const __nv_bfloat16* kr = k_cache + (size_t)row * Lmax * D;
     const float* W = w_k + (size_t)kvh * dg * D;
 
     for (int j = j_first + (int)blockIdx.x; j < NB; j += chunks) {
-        const int t0 = j * blk;
-        const int n = min(blk, L - t0);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int t = rsub; t < n; t += kRowsPerPass) {
-            const uint4 v = *reinterpret_cast<const uint4*>(kr + (size_t)(t0 + t) * D + cpart * 8);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        pool_block_mean<D, BLK>(kr + (size_t)j * BLK * D, min(BLK, L - j * BLK), sm);
+        float pv[D / 32];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                acc[2 * u] += __uint_as_float(w[u] << 16);
-                acc[2 * u + 1] += __uint_as_float(w[u] & 0xffff0000u);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) red[rsub][cpart * 8 + u] = acc[u];
-        __syncthreads();
-        if (tid < D) {
-            float s = 0.f;
-#pragma unroll
-            for (int r = 0; r < kRowsPerPass; ++r) s += red[r][tid];
-            pooled[tid] = s / (float)n;
-        }
-        __syncthreads();
-        constexpr int kVec = D / 32;
-        float pv[kVec];
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) pv[u] = pooled[lane * kVec + u];
-        for (int e = warp; e < dg; e += kThreads / 32) {
-            const float* we = W + (size_t)e * D + lane * kVec;
-            float d = 0.f;
-            if constexpr (kVec == 4) {
-                const float4 wv = *reinterpret_cast<const float4*>(we);
-                d = wv.x * pv[0] + wv.y * pv[1] + wv.z * pv[2] + wv.w * pv[3];
-            } else {
-                const float2 wv = *reinterpret_cast<const float2*>(we);
-                d = wv.x * pv[0] + wv.y * pv[1];
-            }
-            d = warp_sum(d);
-            if (lane == 0) kpool[((size_t)row * NBmax + j) * dg + e] = d;
-        }
-        __syncthreads();  // red / pooled are reused by the next block
+        for (int u = 0; u < D / 32; ++u) pv[u] = sm.pooled[lane * (D / 32) + u];
+        float* dst = kpool + ((size_t)row * NBmax + j) * dg;
+        warp_matvec_rows<D>(W, pv, warp, dg, kThreads / 32, [&](int e, float x) { dst[e] = x; });
+        __syncthreads();  // sm is reused by the next block
     }
 }
 
@@ -96,12 +58,14 @@ cudaError_t launch_kpool_update(const Shape& s, const void* k_cache, const float
     if (upd_start) chunks = 1 + (chunks > 1);  // a decode refresh touches one block, rarely two
     const dim3 grid(chunks, rows);
     const auto* k = static_cast<const __nv_bfloat16*>(k_cache);
-    if (s.D == 128)
-        kpool_update_kernel<128><<<grid, kThreads, 0, stream>>>(k, w_k, seq_lens, upd_start, kpool, s.Hkv, s.Lmax,
-                                                               s.blk, s.dg, s.NBmax, chunks);
-    else
-        kpool_update_kernel<64><<<grid, kThreads, 0, stream>>>(k, w_k, seq_lens, upd_start, kpool, s.Hkv, s.Lmax,
-                                                              s.blk, s.dg, s.NBmax, chunks);
+#define SEER_KPOOL(D_, B_)                                                                                       \
+    kpool_update_kernel<D_, B_><<<grid, kThreads, 0, stream>>>(k, w_k, seq_lens, upd_start, kpool, s.Hkv, s.Lmax, \
+                                                               s.dg, s.NBmax, chunks)
+    if (s.D == 128 && s.blk == 64) SEER_KPOOL(128, 64);
+    else if (s.D == 128) SEER_KPOOL(128, 128);
+    else if (s.blk == 64) SEER_KPOOL(64, 64);
+    else SEER_KPOOL(64, 128);
+#undef SEER_KPOOL
     return cudaGetLastError();
 }
 

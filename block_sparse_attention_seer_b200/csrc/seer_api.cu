@@ -8,6 +8,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 
 #include "seer.h"
 #include "seer_launch.h"
@@ -58,7 +59,13 @@ seer_status check_dims(const seer_dims* d, Shape& s) {
     return SEER_OK;
 }
 
-seer_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SEER_OK : SEER_ERR_CUDA; }
+thread_local char g_last_error[256] = "no error";
+
+seer_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return SEER_OK;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return SEER_ERR_CUDA;
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -173,6 +180,59 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
     return from_cuda(seer::launch_combine(s, o_part, lse_part, num_splits, out, lse_out, stream));
 }
 
+seer_status seer_decode_step_workspace_size(const seer_dims* dims, int32_t budget_tokens, size_t* bytes) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!bytes || budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    *bytes = seer::step_workspace_layout(s, budget_tokens / s.blk, nsm).total;
+    return SEER_OK;
+}
+
+seer_status seer_decode_step(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                             const float* w_q, const float* w_k, const int32_t* seq_lens, const int32_t* upd_start,
+                             int32_t budget_tokens, float sm_scale, float* kpool, int32_t* block_idx,
+                             int32_t* num_selected, void* out, float* lse_out, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !k_cache || !v_cache || !w_q || !w_k || !seq_lens || !kpool || !block_idx || !num_selected || !out ||
+        !workspace)
+        return SEER_ERR_INVALID_ARG;
+    if (budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(w_q, 16) ||
+        !aligned(w_k, 16) || !aligned(kpool, 16) || !aligned(workspace, 256) || !aligned(out, 2))
+        return SEER_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
+    if (s.NBmax > 16384) return SEER_ERR_UNSUPPORTED;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    if (workspace_bytes < seer::step_workspace_layout(s, budget_tokens / s.blk, nsm).total)
+        return SEER_ERR_INVALID_ARG;
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, k_cache, s) || !encode_cache_map(&tmv, v_cache, s)) return SEER_ERR_CUDA;
+    seer::StepLaunch a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.w_q = w_q;
+    a.w_k = w_k;
+    a.seq_lens = seq_lens;
+    a.upd_start = upd_start;
+    a.budget_tokens = budget_tokens;
+    a.sm_scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
+    a.kpool = kpool;
+    a.block_idx = block_idx;
+    a.num_selected = num_selected;
+    a.out = out;
+    a.lse_out = lse_out;
+    a.workspace = workspace;
+    return from_cuda(seer::launch_decode_step(s, a, tmk, tmv, nsm, stream));
+}
+
 seer_status seer_default_num_splits(int32_t kmax, int32_t* num_splits) {
     if (kmax < 1 || !num_splits) return SEER_ERR_INVALID_ARG;
     const int nsm = device_sm_count();
@@ -180,6 +240,24 @@ seer_status seer_default_num_splits(int32_t kmax, int32_t* num_splits) {
     *num_splits = kmax < nsm ? kmax : nsm;
     return SEER_OK;
 }
+
+seer_status seer_decode_wait_failures(uint32_t* count, int32_t reset) {
+    if (!count) return SEER_ERR_INVALID_ARG;
+    unsigned int c = 0;
+    if (seer::read_decode_wait_failures(&c, reset != 0) != cudaSuccess) return SEER_ERR_CUDA;
+    *count = c;
+    return SEER_OK;
+}
+
+seer_status seer_wait_selftest(int64_t limit_ns, int32_t* timed_out) {
+    if (!timed_out || limit_ns < 0 || limit_ns > 2000000000LL) return SEER_ERR_INVALID_ARG;
+    int r = -1;
+    if (seer::run_wait_selftest((unsigned long long)limit_ns, &r) != cudaSuccess) return SEER_ERR_CUDA;
+    *timed_out = r;
+    return SEER_OK;
+}
+
+const char* seer_last_error_string(void) { return g_last_error; }
 
 const char* seer_status_string(seer_status status) {
     switch (status) {

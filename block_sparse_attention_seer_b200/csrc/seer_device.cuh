@@ -53,15 +53,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for the phase of `parity` to complete; false after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of `parity` to complete; false once `limit_ns` has passed.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -153,6 +153,43 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
+}
+
+// out[e] = W[e, :] . v for the rows e = first, first + stride, ... < end, one
+// warp per row with 8 rows in flight: each lane holds D/32 entries of v
+// (vd) and reads the matching 16- or 8-byte piece of each W row (coalesced
+// across the warp). Lane 0 of the warp returns the dot through `sink`.
+template <int D, typename Sink>
+__device__ __forceinline__ void warp_matvec_rows(const float* __restrict__ W, const float (&vd)[D / 32], int first,
+                                                 int end, int stride, Sink sink) {
+    constexpr int kVec = D / 32;
+    const int lane = threadIdx.x & 31;
+    for (int e0 = first; e0 < end; e0 += 8 * stride) {
+        float d[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * stride;
+            d[u] = 0.f;
+            if (e < end) {
+                const float* we = W + (size_t)e * D + lane * kVec;
+                if constexpr (kVec == 4) {
+                    const float4 w = *reinterpret_cast<const float4*>(we);
+                    d[u] = w.x * vd[0] + w.y * vd[1] + w.z * vd[2] + w.w * vd[3];
+                } else {
+                    const float2 w = *reinterpret_cast<const float2*>(we);
+                    d[u] = w.x * vd[0] + w.y * vd[1];
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float x = d[u];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            const int e = e0 + u * stride;
+            if (lane == 0 && e < end) sink(e, x);
+        }
+    }
 }
 
 // Named barrier over `threads` threads (a multiple of 32), id 1..15.

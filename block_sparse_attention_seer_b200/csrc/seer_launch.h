@@ -41,6 +41,39 @@ cudaError_t launch_sparse_decode(const Shape& s, const DecodeLaunch& a, const CU
 // Number of CTAs the decode kernel runs for these arguments (1 per SM at most).
 int sparse_decode_ctas(const Shape& s, int kmax, int num_splits, int num_sms);
 
+// The whole decode step in one cooperative launch (sparse_decode.cu).
+struct StepLaunch {
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const float* w_q;
+    const float* w_k;
+    const int32_t* seq_lens;
+    const int32_t* upd_start;  // NULL: refresh the last block only
+    int budget_tokens;
+    float sm_scale;  // resolved (> 0)
+    float* kpool;
+    int32_t* block_idx;
+    int32_t* num_selected;
+    void* out;
+    float* lse_out;
+    void* workspace;
+};
+
+// Byte offsets inside the step's workspace.
+struct WorkspaceLayout {
+    size_t grid_bar, row_done, o_part, lse_part, total;
+};
+WorkspaceLayout step_workspace_layout(const Shape& s, int kmax, int num_sms);
+
+cudaError_t launch_decode_step(const Shape& s, const StepLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                               int num_sms, cudaStream_t stream);
+
+// Failure detection: the decode kernel's count of CTAs that gave up on a
+// bounded wait, and a self-test of the bounded wait (synchronous).
+cudaError_t read_decode_wait_failures(unsigned int* count, bool reset);
+cudaError_t run_wait_selftest(unsigned long long limit_ns, int* timed_out);
+
 cudaError_t launch_combine(const Shape& s, const float* o_part, const float* lse_part, int num_splits,
                            void* out, float* lse_out, cudaStream_t stream);
 

@@ -1,4 +1,5 @@
-// sparse_decode.cu -- block-sparse split-KV flash-decode for sm_100a.
+// sparse_decode.cu -- block-sparse split-KV flash-decode for sm_100a, and the
+// whole decode step fused into one cooperative launch.
 //
 // Computes, for every (batch b, KV head kvh) row and each of its G query
 // heads, softmax attention over the valid tokens of the kept KV blocks only:
@@ -11,7 +12,7 @@
 //    to end (kmax positions per row), are cut into P equal contiguous
 //    ranges, one per CTA, so each SM streams the same number of blocks and
 //    its copy pipeline never drains between rows. Each (CTA, row) overlap
-//    produces one partial (o, lse) "slot"; seer_combine merges slots.
+//    produces one partial (o, lse) "slot".
 //  * one producer warp: a single lane issues 2-D TMA tile loads (128-byte
 //    swizzle) of the whole K and V tile of each kept block straight into a
 //    ring of shared-memory stages, with an mbarrier pair per stage; the
@@ -27,18 +28,31 @@
 //  * tokens t >= L_b of the partial last block are masked to -inf and their
 //    V rows zeroed in shared memory before P V (the cache past L_b may hold
 //    anything, NaN included).
-//  * every wait is an mbarrier wait with a time limit; on expiry the CTA
-//    records an error, writes NaN into the slot it was producing and exits
-//    after its own copies have landed.
+//  * every wait is bounded (mbarrier waits and the grid barrier alike); on
+//    expiry the CTA counts a failure, writes NaN into the slot it was
+//    producing and leaves only after its own copies have landed.
+//
+// sparse_decode_kernel (seer_sparse_decode) writes the slots; seer_combine
+// merges them. decode_step_kernel (seer_decode_step) runs the whole step in
+// one cooperative launch:
+//   phase 1, one CTA per row (strided): refresh the pooled-K rows of the open
+//     block(s), project the group's mean query, score the cached pooled keys
+//     (streamed into the idle stage ring by bulk copies), select the kept
+//     blocks -- with the same arithmetic as the separate kernels
+//     (gate_core.cuh), so both paths give bit-identical block lists;
+//   a bounded grid barrier;
+//   phase 2, the decode above; the last CTA to finish a row's slots (an
+//     atomic count per row) merges them into the output in place of
+//     seer_combine, and resets the count for the next call.
 #include <cfloat>
 #include <cmath>
 
-#include "seer_device.cuh"
+#include "gate_core.cuh"
 #include "seer_launch.h"
 
 namespace seer {
 
-// Count of decode CTAs that gave up on a wait (0 in normal operation).
+// Count of CTAs that gave up on a bounded wait (0 in normal operation).
 __device__ unsigned int g_decode_wait_failures = 0;
 
 namespace {
@@ -47,7 +61,10 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kMaxStages = 8;
-constexpr int kSmemLimit = 232448;  // 227 KB of opt-in dynamic shared memory per CTA
+constexpr int kMaxGateStages = 8;
+constexpr int kSmemLimit = 232448;       // 227 KB of opt-in dynamic shared memory per CTA
+constexpr int kGateScratchBytes = 16384;  // phase-1 scratch at the start of the stage ring
+constexpr int kGateChunkBytes = 32768;    // phase-1 bulk copy unit (pooled-K rows)
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -75,12 +92,42 @@ struct Params {
     float scale_log2;  // sm_scale * log2(e)
 };
 
+// Extra arguments of the fused step (phase 1 and the in-kernel merge).
+struct StepParams {
+    const __nv_bfloat16* k_cache;
+    const float* w_q;
+    const float* w_k;
+    const int32_t* upd_start;
+    float* kpool;
+    int32_t* block_idx;     // phase-1 output, phase-2 input
+    int32_t* num_selected;  // idem
+    __nv_bfloat16* out;
+    float* lse_out;
+    unsigned int* grid_bar;  // {arrivals, generation}
+    unsigned int* row_done;  // [rows] finished slots per row
+    int rows, NBmax;
+    int keys_off, chunk_off, n_gate_stages;  // phase-1 layout inside the stage ring
+};
+
+// Shared-memory info words after the per-stage `valid` counts.
+constexpr int kInfoAbort = kMaxStages;      // a wait of this CTA gave up
+constexpr int kInfoMergeRow = kMaxStages + 1;  // this CTA merges the current row
+constexpr int kInfoWords = kMaxStages + 4;
+
 // One row's share of this CTA's range.
 struct Segment {
     int row, b, kvh, L, a0, a1, slot, nslots;
     bool last;  // this CTA holds the end of the row's reserved positions
 };
 
+template <bool kFresh>
+__device__ __forceinline__ int load_i32(const int32_t* p) {
+    // Values written earlier in the same launch by other CTAs bypass L1.
+    if constexpr (kFresh) return __ldcg(p);
+    else return *p;
+}
+
+template <bool kFused>
 __device__ __forceinline__ Segment make_segment(const Params& p, int r, long long g0, long long g1) {
     Segment s;
     const long long rs = (long long)r * p.kmax;
@@ -90,7 +137,7 @@ __device__ __forceinline__ Segment make_segment(const Params& p, int r, long lon
     s.b = r / p.Hkv;
     s.kvh = r - s.b * p.Hkv;
     s.L = clamp_len(p.seq_lens[s.b], p.Lmax);
-    int n = s.L == 0 ? 0 : p.num_selected[r];
+    int n = s.L == 0 ? 0 : load_i32<kFused>(p.num_selected + r);
     n = n < 0 ? 0 : (n > p.kmax ? p.kmax : n);
     s.a0 = i0 < n ? i0 : n;
     s.a1 = i1 < n ? i1 : n;
@@ -111,127 +158,196 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int tok, int d0) {
     return tile + (uint32_t)((d0 >> 6) * (BLK * 128) + tok * 128 + ((((d0 & 63) >> 3) ^ (tok & 7)) << 4));
 }
 
-__device__ __forceinline__ void record_failure(int* abort_flag) {
-    if (atomicExch(abort_flag, 1) == 0) atomicAdd(&g_decode_wait_failures, 1u);
+__device__ __forceinline__ void record_failure(int* info) {
+    if (atomicExch(info + kInfoAbort, 1) == 0) atomicAdd(&g_decode_wait_failures, 1u);
 }
 
-template <int D, int BLK>
-__global__ void __launch_bounds__(kThreads, 1)
-    sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                         const Params p) {
-    using C = Cfg<D, BLK>;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~uintptr_t(1023));
-    const uint32_t sbase = smem_addr(base);
-    float* merge = reinterpret_cast<float*>(base + p.merge_off);
-    int* info = reinterpret_cast<int*>(base + p.info_off);
-    int* abort_flag = info + kMaxStages;
-    const uint32_t bars = sbase + p.bar_off;  // full[0..nst), empty[0..nst), consumer barrier
-    auto bar_full = [&](int st) { return bars + 8u * st; };
-    auto bar_empty = [&](int st) { return bars + 8u * (p.nst + st); };
-    const uint32_t bar_cons = bars + 16u * p.nst;
+// Shared-memory views common to both kernels.
+struct Smem {
+    unsigned char* base;  // 1024-aligned
+    uint32_t sbase;
+    float* merge;
+    int* info;
+    uint32_t bars;
+    int nst;
+    __device__ __forceinline__ uint32_t full(int st) const { return bars + 8u * st; }
+    __device__ __forceinline__ uint32_t empty(int st) const { return bars + 8u * (nst + st); }
+    __device__ __forceinline__ uint32_t cons() const { return bars + 16u * nst; }
+    __device__ __forceinline__ uint32_t gate(int st) const { return bars + 16u * nst + 8u + 8u * st; }
+};
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) {
+    Smem m;
+    m.base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    m.sbase = smem_addr(m.base);
+    m.merge = reinterpret_cast<float*>(m.base + p.merge_off);
+    m.info = reinterpret_cast<int*>(m.base + p.info_off);
+    m.bars = m.sbase + p.bar_off;
+    m.nst = p.nst;
     if (threadIdx.x == 0) {
         for (int st = 0; st < p.nst; ++st) {
-            mbar_init(bar_full(st), 1);
-            mbar_init(bar_empty(st), kConsumerWarps);
+            mbar_init(m.full(st), 1);
+            mbar_init(m.empty(st), kConsumerWarps);
         }
-        mbar_init(bar_cons, kConsumerThreads);
-        *abort_flag = 0;
+        mbar_init(m.cons(), kConsumerThreads);
+        for (int st = 0; st < kMaxGateStages; ++st) mbar_init(m.gate(st), 1);
+        for (int i = 0; i < kInfoWords; ++i) m.info[i] = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    return m;
+}
 
-    const long long g0 = (long long)blockIdx.x * p.V / p.P;
-    const long long g1 = (long long)(blockIdx.x + 1) * p.V / p.P;
-    const int r_begin = (int)(g0 / p.kmax);
+// All 256 consumer threads meet (bounded); false if the wait gave up.
+__device__ __forceinline__ bool consumer_sync(const Smem& m, uint32_t& cph) {
+    mbar_arrive(m.cons());
+    const bool ok = mbar_wait(m.cons(), cph);
+    cph ^= 1u;
+    if (!ok) record_failure(m.info);
+    return ok;
+}
 
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer warp
-        if (lane == 0) {
-            prefetch_tensor_map(&tmK);
-            prefetch_tensor_map(&tmV);
-        }
-        const uint64_t policy = l2_policy_evict_first();
-        int st = 0;
-        uint32_t ph = 0;
-        long long issued = 0;
-        bool ok = true;
-        for (int r = r_begin; ok && (long long)r * p.kmax < g1; ++r) {
-            const Segment s = make_segment(p, r, g0, g1);
-            if (s.a1 <= s.a0) continue;
-            const int NB = (s.L + BLK - 1) / BLK;
-            const __nv_bfloat16* qsrc = p.q + ((size_t)s.b * p.Hq + (size_t)s.kvh * p.G) * D;
-            const int32_t* list = p.block_idx + (size_t)r * p.kmax;
-            for (int i = s.a0; ok && i < s.a1; i += 32) {
-                const int jl = (i + lane < s.a1) ? list[i + lane] : -1;
-                const int cnt = min(32, s.a1 - i);
-                for (int k = 0; ok && k < cnt; ++k) {
-                    const int j = __shfl_sync(0xffffffffu, jl, k);
-                    const int valid = (j >= 0 && j < NB) ? min(BLK, s.L - j * BLK) : 0;
-                    int good = 1;
-                    if (lane == 0) {
-                        if (!mbar_wait(bar_empty(st), ph ^ 1u)) {
-                            good = 0;
-                            record_failure(abort_flag);
-                        } else {
-                            info[st] = valid;
-                            const bool first = (i + k == s.a0);
-                            const uint32_t fb = bar_full(st);
-                            const uint32_t bytes =
-                                (valid > 0 ? 2u * C::kTileBytes : 0u) + (first ? (uint32_t)(p.G * D * 2) : 0u);
-                            if (bytes) mbar_arrive_expect_tx(fb, bytes);
-                            else mbar_arrive(fb);
-                            const uint32_t stK = sbase + (uint32_t)st * p.stage_bytes;
-                            if (valid > 0) {
-                                const int y = r * p.Lmax + j * BLK;
+// ---------------------------------------------------------------- decode: producer warp
+
+template <int D, int BLK, bool kFused>
+__device__ void decode_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, const Params& p, const Smem& m,
+                                long long g0, long long g1) {
+    using C = Cfg<D, BLK>;
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) {
+        prefetch_tensor_map(tmK);
+        prefetch_tensor_map(tmV);
+    }
+    const uint64_t policy = l2_policy_evict_first();
+    int st = 0;
+    uint32_t ph = 0;
+    long long issued = 0;
+    bool ok = true;
+    for (int r = (int)(g0 / p.kmax); ok && (long long)r * p.kmax < g1; ++r) {
+        const Segment s = make_segment<kFused>(p, r, g0, g1);
+        if (s.a1 <= s.a0) continue;
+        const int NB = (s.L + BLK - 1) / BLK;
+        const __nv_bfloat16* qsrc = p.q + ((size_t)s.b * p.Hq + (size_t)s.kvh * p.G) * D;
+        const int32_t* list = p.block_idx + (size_t)r * p.kmax;
+        for (int i = s.a0; ok && i < s.a1; i += 32) {
+            const int jl = (i + lane < s.a1) ? load_i32<kFused>(list + i + lane) : -1;
+            const int cnt = min(32, s.a1 - i);
+            for (int k = 0; ok && k < cnt; ++k) {
+                const int j = __shfl_sync(0xffffffffu, jl, k);
+                const int valid = (j >= 0 && j < NB) ? min(BLK, s.L - j * BLK) : 0;
+                int good = 1;
+                if (lane == 0) {
+                    if (!mbar_wait(m.empty(st), ph ^ 1u)) {
+                        good = 0;
+                        record_failure(m.info);
+                    } else {
+                        m.info[st] = valid;
+                        const bool first = (i + k == s.a0);
+                        const uint32_t fb = m.full(st);
+                        const uint32_t bytes =
+                            (valid > 0 ? 2u * C::kTileBytes : 0u) + (first ? (uint32_t)(p.G * D * 2) : 0u);
+                        if (bytes) mbar_arrive_expect_tx(fb, bytes);
+                        else mbar_arrive(fb);
+                        const uint32_t stK = m.sbase + (uint32_t)st * p.stage_bytes;
+                        if (valid > 0) {
+                            const int y = r * p.Lmax + j * BLK;
 #pragma unroll
-                                for (int bx = 0; bx < C::kBoxes; ++bx) {
-                                    tma_load_2d(stK + bx * C::kBoxBytes, &tmK, fb, bx * 64, y, policy);
-                                    tma_load_2d(stK + C::kTileBytes + bx * C::kBoxBytes, &tmV, fb, bx * 64, y,
-                                                policy);
-                                }
+                            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                                tma_load_2d(stK + bx * C::kBoxBytes, tmK, fb, bx * 64, y, policy);
+                                tma_load_2d(stK + C::kTileBytes + bx * C::kBoxBytes, tmV, fb, bx * 64, y, policy);
                             }
-                            if (first) bulk_load(stK + 2 * C::kTileBytes, qsrc, (uint32_t)(p.G * D * 2), fb);
-                            ++issued;
                         }
+                        if (first) bulk_load(stK + 2 * C::kTileBytes, qsrc, (uint32_t)(p.G * D * 2), fb);
+                        ++issued;
                     }
-                    ok = __shfl_sync(0xffffffffu, good, 0) != 0;
-                    if (ok && ++st == p.nst) {
-                        st = 0;
-                        ph ^= 1u;
-                    }
+                }
+                ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+                if (ok && ++st == p.nst) {
+                    st = 0;
+                    ph ^= 1u;
                 }
             }
         }
-        if (lane == 0) {
-            // Tail: the producer warp leaves only once every copy it issued has
-            // landed -- normally by seeing the consumers release the last stages,
-            // after a failed wait by seeing the copies complete.
-            for (long long it = (issued > p.nst ? issued - p.nst : 0); it < issued; ++it) {
-                const int s_it = (int)(it % p.nst);
-                const uint32_t par = (uint32_t)((it / p.nst) & 1);
-                if (!ok || !mbar_wait(bar_empty(s_it), par)) (void)mbar_wait(bar_full(s_it), par);
-            }
-        }
-        return;
     }
+    if (lane == 0) {
+        // Tail: the producer warp leaves only once every copy it issued has
+        // landed -- normally by seeing the consumers release the last stages,
+        // after a failed wait by seeing the copies complete.
+        for (long long it = (issued > p.nst ? issued - p.nst : 0); it < issued; ++it) {
+            const int s_it = (int)(it % p.nst);
+            const uint32_t par = (uint32_t)((it / p.nst) & 1);
+            if (!ok || !mbar_wait(m.empty(s_it), par)) (void)mbar_wait(m.full(s_it), par);
+        }
+    }
+}
 
-    // ---------------------------------------------------------------- consumer warps
+// ---------------------------------------------------------------- decode: in-kernel merge (fused step)
+
+// The last CTA to finish a slot of row `s.row` merges all of the row's slots
+// into out / lse_out (log-sum-exp weights) and resets the row's count.
+template <int D>
+__device__ void merge_row_if_last(const Params& p, const StepParams& f, const Smem& m, const Segment& s,
+                                  uint32_t& cph) {
+    const int ctid = threadIdx.x;
+    __threadfence();  // this CTA's slot writes before its count
+    if (!consumer_sync(m, cph)) return;
+    if (ctid == 0) {
+        const unsigned int done = atomicAdd(f.row_done + s.row, 1u) + 1u;
+        m.info[kInfoMergeRow] = (done == (unsigned int)s.nslots);
+    }
+    if (!consumer_sync(m, cph)) return;
+    if (!m.info[kInfoMergeRow]) return;
+    __threadfence();  // other CTAs' slots, published before their counts
+    const size_t head0 = (size_t)s.b * p.Hq + (size_t)s.kvh * p.G;
+    const int ns = s.nslots;
+    float* w = m.merge;  // [G][ns] normalised slot weights (the merge area is free here)
+    if (ctid < p.G) {
+        const float* l = p.lse_part + (head0 + ctid) * p.S;
+        float M = -INFINITY;
+        for (int k = 0; k < ns; ++k) M = fmaxf(M, __ldcg(l + k));
+        float wsum = 0.f;
+        for (int k = 0; k < ns; ++k) {
+            const float lk = __ldcg(l + k);
+            const float e = (lk == -INFINITY || M == -INFINITY) ? 0.f : expf(lk - M);
+            w[ctid * ns + k] = e;
+            wsum += e;
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        for (int k = 0; k < ns; ++k) w[ctid * ns + k] *= inv;
+        if (f.lse_out) f.lse_out[head0 + ctid] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
+    }
+    if (!consumer_sync(m, cph)) return;
+    for (int idx = ctid; idx < p.G * D; idx += kConsumerThreads) {
+        const int h = idx / D, d = idx - h * D;
+        float acc = 0.f;
+        for (int k = 0; k < ns; ++k) {
+            const float wk = w[h * ns + k];
+            if (wk != 0.f) acc += wk * __ldcg(p.o_part + ((head0 + h) * p.S + k) * D + d);
+        }
+        f.out[(head0 + h) * D + d] = __float2bfloat16(acc);
+    }
+    if (ctid == 0) f.row_done[s.row] = 0u;
+    (void)consumer_sync(m, cph);  // the weights area is reused by the next segment
+}
+
+// ---------------------------------------------------------------- decode: consumer warps
+
+template <int D, int BLK, bool kFused>
+__device__ void decode_consumers(const Params& p, const StepParams& f, const Smem& m, long long g0, long long g1) {
+    using C = Cfg<D, BLK>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ctid = threadIdx.x;                  // 0 .. 255
     const int g = lane >> 2, tig = lane & 3;       // mma fragment coordinates
     const int tbase = warp * C::kTokPerWarp;       // this warp's token slice of each block
-    float* mO = merge;                             // [8][G][D]
-    float* mM = merge + kConsumerWarps * p.G * D;  // [8][G]
+    float* mO = m.merge;                           // [8][G][D]
+    float* mM = m.merge + kConsumerWarps * p.G * D;  // [8][G]
     float* mL = mM + kConsumerWarps * p.G;         // [8][G]
     int st = 0;
     uint32_t ph = 0, cph = 0;
     bool ok = true;
 
-    for (int r = r_begin; ok && (long long)r * p.kmax < g1; ++r) {
-        const Segment s = make_segment(p, r, g0, g1);
+    for (int r = (int)(g0 / p.kmax); ok && (long long)r * p.kmax < g1; ++r) {
+        const Segment s = make_segment<kFused>(p, r, g0, g1);
         const size_t head0 = (size_t)s.b * p.Hq + (size_t)s.kvh * p.G;
         if (s.a1 > s.a0) {
             float m_run = -INFINITY, l_run = 0.f;
@@ -241,17 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t qa[C::kKSteps][2];
 
             for (int i = s.a0; i < s.a1; ++i) {
-                if (!mbar_wait(bar_full(st), ph)) {
-                    record_failure(abort_flag);
+                if (!mbar_wait(m.full(st), ph)) {
+                    record_failure(m.info);
                     ok = false;
                     break;
                 }
-                const int valid = info[st];
-                const uint32_t stK = sbase + (uint32_t)st * p.stage_bytes;
+                const int valid = m.info[st];
+                const uint32_t stK = m.sbase + (uint32_t)st * p.stage_bytes;
                 const uint32_t stV = stK + C::kTileBytes;
                 if (i == s.a0) {
-                    const __nv_bfloat16* qs =
-                        reinterpret_cast<const __nv_bfloat16*>(base + (size_t)st * p.stage_bytes + 2 * C::kTileBytes);
+                    const __nv_bfloat16* qs = reinterpret_cast<const __nv_bfloat16*>(
+                        m.base + (size_t)st * p.stage_bytes + 2 * C::kTileBytes);
 #pragma unroll
                     for (int kk = 0; kk < C::kKSteps; ++kk) {
                         qa[kk][0] = g < p.G ? *reinterpret_cast<const uint32_t*>(qs + g * D + kk * 16 + 2 * tig) : 0u;
@@ -363,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (wrote) fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_empty(st));
+                if (lane == 0) mbar_arrive(m.empty(st));
                 if (++st == p.nst) {
                     st = 0;
                     ph ^= 1u;
@@ -387,48 +503,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int dt = 0; dt < C::kDTiles; ++dt)
                     *reinterpret_cast<float2*>(dst + dt * 8) = make_float2(o[dt][0], o[dt][1]);
             }
-            mbar_arrive(bar_cons);
-            if (!mbar_wait(bar_cons, cph)) {
-                record_failure(abort_flag);
-                ok = false;
-            }
-            cph ^= 1u;
-            if (ok) {
-                for (int idx = ctid; idx < p.G * D; idx += kConsumerThreads) {
-                    const int h = idx / D, d = idx - h * D;
-                    float M = -INFINITY;
+            if (!(ok = consumer_sync(m, cph))) break;
+            for (int idx = ctid; idx < p.G * D; idx += kConsumerThreads) {
+                const int h = idx / D, d = idx - h * D;
+                float M = -INFINITY;
 #pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mM[w * p.G + h]);
-                    float* lse_dst = p.lse_part + (head0 + h) * p.S + s.slot;
-                    if (M == -INFINITY) {
-                        if (d == 0) *lse_dst = -INFINITY;
-                        continue;
-                    }
-                    float wsum = 0.f, acc = 0.f;
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mM[w * p.G + h]);
+                float* lse_dst = p.lse_part + (head0 + h) * p.S + s.slot;
+                if (M == -INFINITY) {
+                    if (d == 0) *lse_dst = -INFINITY;
+                    continue;
+                }
+                float wsum = 0.f, acc = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w) {
-                        const float mw = mM[w * p.G + h];
-                        if (mw != -INFINITY) {
-                            const float e = exp2f(mw - M);
-                            wsum += e * mL[w * p.G + h];
-                            acc += e * mO[(size_t)(w * p.G + h) * D + d];
-                        }
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float mw = mM[w * p.G + h];
+                    if (mw != -INFINITY) {
+                        const float e = exp2f(mw - M);
+                        wsum += e * mL[w * p.G + h];
+                        acc += e * mO[(size_t)(w * p.G + h) * D + d];
                     }
-                    p.o_part[((head0 + h) * p.S + s.slot) * D + d] = acc / wsum;
-                    if (d == 0) *lse_dst = (M + log2f(wsum)) * kLn2;
                 }
-                // the merge area is reused by the next segment
-                mbar_arrive(bar_cons);
-                if (!mbar_wait(bar_cons, cph)) {
-                    record_failure(abort_flag);
-                    ok = false;
-                }
-                cph ^= 1u;
+                p.o_part[((head0 + h) * p.S + s.slot) * D + d] = acc / wsum;
+                if (d == 0) *lse_dst = (M + log2f(wsum)) * kLn2;
             }
+            // the merge area is reused by the next segment
+            if (!(ok = consumer_sync(m, cph))) break;
         } else if (ctid < p.G) {
             p.lse_part[(head0 + ctid) * p.S + s.slot] = -INFINITY;  // no kept block in this piece
         }
-        if (s.last) {
+        if constexpr (kFused) {
+            merge_row_if_last<D>(p, f, m, s, cph);
+            ok = m.info[kInfoAbort] == 0;
+        } else if (s.last) {
             const int rest = p.S - s.nslots;
             for (int idx = ctid; idx < p.G * rest; idx += kConsumerThreads) {
                 const int h = idx / rest;
@@ -437,6 +544,197 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 }
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registers as 12: <= 168 each
+    sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const Params p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const Smem m = setup_smem(smem_raw, p);
+    const long long g0 = (long long)blockIdx.x * p.V / p.P;
+    const long long g1 = (long long)(blockIdx.x + 1) * p.V / p.P;
+    if ((threadIdx.x >> 5) == kConsumerWarps) decode_producer<D, BLK, false>(&tmK, &tmV, p, m, g0, g1);
+    else decode_consumers<D, BLK, false>(p, StepParams{}, m, g0, g1);
+}
+
+// ---------------------------------------------------------------- fused step: phase 1 (gate + select)
+
+template <int D, int DG>
+struct GateScratch {
+    PoolSmem<D> pool;
+    SelectSmem<kThreads> sel;
+    alignas(16) float qbar[D];
+    alignas(16) float qg[DG];
+    alignas(16) float kp_new[DG];
+};
+static_assert(sizeof(GateScratch<128, 128>) <= kGateScratchBytes, "phase-1 scratch");
+
+template <int D, int BLK, int DG>
+__device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) {
+    constexpr int kWarps = kThreads / 32;
+    constexpr int kVecG = DG / 32;
+    constexpr int kChunkRows = kGateChunkBytes / (DG * 4);
+    using Vec = GateVec<DG>;
+    GateScratch<D, DG>& sm = *reinterpret_cast<GateScratch<D, DG>*>(m.base);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(m.base + f.keys_off);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
+    int chunk_it = 0;  // bulk-copy stages used so far (same count on every thread)
+
+    for (int r = blockIdx.x; r < f.rows; r += gridDim.x) {
+        const int b = r / p.Hkv, kvh = r - b * p.Hkv;
+        const int L = clamp_len(p.seq_lens[b], p.Lmax);
+        const int NB = (L + BLK - 1) / BLK;
+        const int kb = p.kmax < NB ? p.kmax : NB;
+        int js = NB;  // first block whose pooled key is refreshed
+        if (NB > 0) {
+            int st0 = f.upd_start ? f.upd_start[b] : L - 1;
+            st0 = st0 < 0 ? 0 : st0;
+            js = min(st0 / BLK, NB);
+        }
+        const int ncand = NB - 1;
+        const bool scored = kb - 1 > 0 && kb - 1 < ncand;  // otherwise the choice needs no score
+        const int nscan = scored ? min(js, ncand) : 0;      // cached rows to score
+        const int nchunks = (nscan + kChunkRows - 1) / kChunkRows;
+        float* kp_row = f.kpool + (size_t)r * f.NBmax * DG;
+        auto chunk_dst = [&](int stage) { return m.sbase + (uint32_t)(f.chunk_off + stage * kGateChunkBytes); };
+        auto issue = [&](int i) {  // chunk i of this row into stage (chunk_it + i) % n
+            const int stage = (chunk_it + i) % f.n_gate_stages;
+            const int rows_i = min(kChunkRows, nscan - i * kChunkRows);
+            const uint32_t bytes = (uint32_t)(rows_i * DG * 4);
+            mbar_arrive_expect_tx(m.gate(stage), bytes);
+            bulk_load(chunk_dst(stage), kp_row + (size_t)i * kChunkRows * DG, bytes, m.gate(stage));
+        };
+        if (tid == 0)
+            for (int i = 0; i < min(f.n_gate_stages, nchunks); ++i) issue(i);
+        // projected query of the group
+        group_query_mean<D>(p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G) * D, p.G, sm.qbar);
+        __syncthreads();
+        {
+            float qv[D / 32];
+#pragma unroll
+            for (int u = 0; u < D / 32; ++u) qv[u] = sm.qbar[lane * (D / 32) + u];
+            warp_matvec_rows<D>(f.w_q + (size_t)kvh * DG * D, qv, warp, DG, kWarps,
+                                [&](int e, float x) { sm.qg[e] = x; });
+        }
+        __syncthreads();
+        float gv[kVecG];
+#pragma unroll
+        for (int u = 0; u < kVecG; ++u) gv[u] = sm.qg[lane * kVecG + u];
+        // refresh the pooled keys of the open block(s); score them if they compete
+        const __nv_bfloat16* krow = f.k_cache + (size_t)r * p.Lmax * D;
+        for (int j = js; j < NB; ++j) {
+            pool_block_mean<D, BLK>(krow + (size_t)j * BLK * D, min(BLK, L - j * BLK), sm.pool);
+            float pv[D / 32];
+#pragma unroll
+            for (int u = 0; u < D / 32; ++u) pv[u] = sm.pool.pooled[lane * (D / 32) + u];
+            warp_matvec_rows<D>(f.w_k + (size_t)kvh * DG * D, pv, warp, DG, kWarps, [&](int e, float x) {
+                kp_row[(size_t)j * DG + e] = x;
+                sm.kp_new[e] = x;
+            });
+            __syncthreads();
+            if (scored && j < ncand && warp == 0) {
+                const float d = gate_dot<DG>(reinterpret_cast<const Vec*>(sm.kp_new)[lane], gv);
+                if (lane == 0) keys[j] = order_key(d * inv_sqrt_dg);
+            }
+            __syncthreads();
+        }
+        // score the cached rows as their chunks land
+        for (int i = 0; i < nchunks; ++i) {
+            const int stage = (chunk_it + i) % f.n_gate_stages;
+            const uint32_t par = (uint32_t)(((chunk_it + i) / f.n_gate_stages) & 1);
+            if (!mbar_wait(m.gate(stage), par)) record_failure(m.info);
+            const Vec* rows_v = reinterpret_cast<const Vec*>(m.base + f.chunk_off + stage * kGateChunkBytes) + lane;
+            const int j0 = i * kChunkRows;
+            const int nrows = min(kChunkRows, nscan - j0);
+            for (int jr = warp; jr < nrows; jr += kWarps) {
+                const float d = gate_dot<DG>(rows_v[(size_t)jr * 32], gv);
+                if (lane == 0) keys[j0 + jr] = order_key(d * inv_sqrt_dg);
+            }
+            fence_proxy_async_smem();  // these generic reads of the stage precede its next bulk copy
+            __syncthreads();
+            if (tid == 0 && i + f.n_gate_stages < nchunks) issue(i + f.n_gate_stages);
+        }
+        chunk_it += nchunks;
+        __syncthreads();
+        if (tid == 0) f.num_selected[r] = kb;
+        select_row<kThreads>(keys, NB, p.kmax, f.block_idx + (size_t)r * p.kmax, sm.sel);
+        fence_proxy_async_smem();
+        __syncthreads();  // scratch and keys are reused by the next row
+    }
+}
+
+// Bounded barrier over every CTA of a cooperative launch: {count, generation}
+// in global memory, left at count 0 for the next call. False if it gave up.
+__device__ bool grid_barrier(unsigned int* bar, const Smem& m) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        unsigned int gen;
+        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+        const unsigned int arrived = atomicAdd(bar, 1u);
+        bool ok = true;
+        if (arrived == gridDim.x - 1) {
+            atomicExch(bar, 0u);
+            __threadfence();
+            atomicAdd(bar + 1, 1u);
+        } else {
+            const uint64_t t0 = global_timer_ns();
+            while (true) {
+                unsigned int now;
+                asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(now) : "l"(bar + 1) : "memory");
+                if (now != gen) break;
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        if (!ok) record_failure(m.info);
+    }
+    __syncthreads();
+    return m.info[kInfoAbort] == 0;
+}
+
+template <int D, int BLK, int DG>
+__global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registers as 12: <= 168 each
+    decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const Params p, const StepParams f) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const Smem m = setup_smem(smem_raw, p);
+    if (threadIdx.x == 0) {
+        prefetch_tensor_map(&tmK);
+        prefetch_tensor_map(&tmV);
+    }
+    gate_phase<D, BLK, DG>(p, f, m);
+    fence_proxy_async_smem();  // phase-1 use of the ring precedes phase-2 copies into it
+    grid_barrier(f.grid_bar, m);
+    if ((int)blockIdx.x >= p.P) return;  // more SMs than decode ranges
+    const long long g0 = (long long)blockIdx.x * p.V / p.P;
+    const long long g1 = (long long)(blockIdx.x + 1) * p.V / p.P;
+    if ((threadIdx.x >> 5) == kConsumerWarps) decode_producer<D, BLK, true>(&tmK, &tmV, p, m, g0, g1);
+    else decode_consumers<D, BLK, true>(p, f, m, g0, g1);
+}
+
+// One CTA waits, with the given limit, on an mbarrier that nothing ever
+// arrives at; the wait must give up and report it.
+__device__ int g_wait_selftest_result = -1;
+
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool completed = mbar_wait(smem_addr(&bar), 0u, limit_ns);
+    __syncthreads();
+    if (threadIdx.x == 0) g_wait_selftest_result = completed ? 0 : 1;
+}
+
+// ---------------------------------------------------------------- host side
 
 struct Layout {
     int nst, stage_bytes, merge_off, info_off, bar_off, total;
@@ -448,28 +746,19 @@ Layout make_layout(int G) {
     Layout l;
     l.stage_bytes = (2 * C::kTileBytes + G * D * 2 + 1023) / 1024 * 1024;
     const int merge_bytes = kConsumerWarps * G * D * 4 + 2 * kConsumerWarps * G * 4;
-    const int tail = merge_bytes + (kMaxStages + 4) * 4 + (2 * kMaxStages + 2) * 8 + 64;
+    const int bar_bytes = (2 * kMaxStages + 1 + kMaxGateStages) * 8;
+    const int tail = merge_bytes + kInfoWords * 4 + bar_bytes + 64;
     int nst = (kSmemLimit - 1024 - tail) / l.stage_bytes;
     l.nst = nst > kMaxStages ? kMaxStages : nst;
     l.merge_off = l.nst * l.stage_bytes;
     l.info_off = (l.merge_off + merge_bytes + 15) / 16 * 16;
-    l.bar_off = (l.info_off + (kMaxStages + 4) * 4 + 15) / 16 * 16;
-    l.total = l.bar_off + (2 * l.nst + 2) * 8 + 1024;  // + slack for the 1024-byte alignment
+    l.bar_off = (l.info_off + kInfoWords * 4 + 15) / 16 * 16;
+    l.total = l.bar_off + bar_bytes + 1024;  // + slack for the 1024-byte alignment
     return l;
 }
 
 template <int D, int BLK>
-cudaError_t launch_impl(const Shape& s, const DecodeLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                        int num_sms, cudaStream_t stream) {
-    const Layout l = make_layout<D, BLK>(s.G);
-    if (l.nst < 2) return cudaErrorInvalidConfiguration;
-    static bool attr_done = false;  // set once per template instance (benign race)
-    if (!attr_done) {
-        cudaError_t e =
-            cudaFuncSetAttribute(sparse_decode_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+Params make_params(const Shape& s, const DecodeLaunch& a, const Layout& l, int P) {
     Params p;
     p.q = static_cast<const __nv_bfloat16*>(a.q);
     p.seq_lens = a.seq_lens;
@@ -484,18 +773,144 @@ cudaError_t launch_impl(const Shape& s, const DecodeLaunch& a, const CUtensorMap
     p.Lmax = s.Lmax;
     p.kmax = a.kmax;
     p.S = a.num_splits;
-    p.P = sparse_decode_ctas(s, a.kmax, a.num_splits, num_sms);
+    p.P = P;
     p.nst = l.nst;
     p.stage_bytes = l.stage_bytes;
     p.merge_off = l.merge_off;
     p.info_off = l.info_off;
     p.bar_off = l.bar_off;
     p.scale_log2 = a.sm_scale * kLog2e;
+    return p;
+}
+
+template <typename K>
+cudaError_t allow_big_smem(K kernel) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+}
+
+template <int D, int BLK>
+cudaError_t launch_impl(const Shape& s, const DecodeLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                        int num_sms, cudaStream_t stream) {
+    const Layout l = make_layout<D, BLK>(s.G);
+    if (l.nst < 2) return cudaErrorInvalidConfiguration;
+    static bool attr_done = false;  // once per template instance (benign race)
+    if (!attr_done) {
+        cudaError_t e = allow_big_smem(sparse_decode_kernel<D, BLK>);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    const Params p = make_params<D, BLK>(s, a, l, sparse_decode_ctas(s, a.kmax, a.num_splits, num_sms));
     sparse_decode_kernel<D, BLK><<<p.P, kThreads, l.total, stream>>>(tmK, tmV, p);
     return cudaGetLastError();
 }
 
+int step_num_splits(const Shape& s, int kmax, int num_sms) {
+    const long long V = (long long)s.B * s.Hkv * kmax;
+    long long P = num_sms < V ? num_sms : V;
+    return (int)(kmax < P ? kmax : P);
+}
+
+template <int D, int BLK, int DG>
+cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                      int num_sms, cudaStream_t stream) {
+    const Layout l = make_layout<D, BLK>(s.G);
+    if (l.nst < 2) return cudaErrorInvalidConfiguration;
+    const int keys_bytes = (s.NBmax * 4 + 1023) / 1024 * 1024;
+    const int ring = l.nst * l.stage_bytes;
+    const int n_gate = (ring - kGateScratchBytes - keys_bytes) / kGateChunkBytes;
+    if (n_gate < 1) return cudaErrorInvalidConfiguration;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = allow_big_smem(decode_step_kernel<D, BLK, DG>);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    const int kmax = a.budget_tokens / s.blk;
+    const long long V = (long long)s.B * s.Hkv * kmax;
+    const int P = (int)(num_sms < V ? num_sms : V);
+    const int S = step_num_splits(s, kmax, num_sms);
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    WorkspaceLayout wl = step_workspace_layout(s, kmax, num_sms);
+
+    DecodeLaunch d;
+    d.q = a.q;
+    d.seq_lens = a.seq_lens;
+    d.block_idx = a.block_idx;
+    d.num_selected = a.num_selected;
+    d.o_part = reinterpret_cast<float*>(ws + wl.o_part);
+    d.lse_part = reinterpret_cast<float*>(ws + wl.lse_part);
+    d.kmax = kmax;
+    d.num_splits = S;
+    d.sm_scale = a.sm_scale;
+    const Params p = make_params<D, BLK>(s, d, l, P);
+
+    StepParams f;
+    f.k_cache = static_cast<const __nv_bfloat16*>(a.k_cache);
+    f.w_q = a.w_q;
+    f.w_k = a.w_k;
+    f.upd_start = a.upd_start;
+    f.kpool = a.kpool;
+    f.block_idx = a.block_idx;
+    f.num_selected = a.num_selected;
+    f.out = static_cast<__nv_bfloat16*>(a.out);
+    f.lse_out = a.lse_out;
+    f.grid_bar = reinterpret_cast<unsigned int*>(ws + wl.grid_bar);
+    f.row_done = reinterpret_cast<unsigned int*>(ws + wl.row_done);
+    f.rows = s.B * s.Hkv;
+    f.NBmax = s.NBmax;
+    f.keys_off = kGateScratchBytes;
+    f.chunk_off = kGateScratchBytes + keys_bytes;
+    f.n_gate_stages = n_gate > kMaxGateStages ? kMaxGateStages : n_gate;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms, 1, 1);  // every SM: phase 1 spreads rows over all of them
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = l.total;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_step_kernel<D, BLK, DG>, tmK, tmV, p, f);
+    if (e != cudaSuccess) (void)cudaGetLastError();  // a rejected launch must not leak into the next call
+    return e;
+}
+
 }  // namespace
+
+WorkspaceLayout step_workspace_layout(const Shape& s, int kmax, int num_sms) {
+    WorkspaceLayout w;
+    const size_t rows = (size_t)s.B * s.Hkv;
+    const size_t S = (size_t)step_num_splits(s, kmax, num_sms);
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    w.grid_bar = 0;
+    w.row_done = 256;
+    w.o_part = up(w.row_done + rows * 4);
+    w.lse_part = up(w.o_part + (size_t)s.B * s.Hq * S * s.D * 4);
+    w.total = up(w.lse_part + (size_t)s.B * s.Hq * S * 4);
+    return w;
+}
+
+cudaError_t read_decode_wait_failures(unsigned int* count, bool reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(count, g_decode_wait_failures, sizeof(unsigned int));
+    if (e != cudaSuccess || !reset) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_decode_wait_failures, &zero, sizeof(unsigned int));
+}
+
+cudaError_t run_wait_selftest(unsigned long long limit_ns, int* timed_out) {
+    const int unset = -1;
+    cudaError_t e = cudaMemcpyToSymbol(g_wait_selftest_result, &unset, sizeof(int));
+    if (e != cudaSuccess) return e;
+    wait_selftest_kernel<<<1, 32>>>(limit_ns);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return e;
+    int r = -1;
+    if ((e = cudaMemcpyFromSymbol(&r, g_wait_selftest_result, sizeof(int))) != cudaSuccess) return e;
+    *timed_out = r;
+    return cudaSuccess;
+}
 
 int sparse_decode_ctas(const Shape& s, int kmax, int num_splits, int num_sms) {
     const long long V = (long long)s.B * s.Hkv * kmax;
@@ -511,6 +926,22 @@ cudaError_t launch_sparse_decode(const Shape& s, const DecodeLaunch& a, const CU
     if (s.D == 128 && s.blk == 128) return launch_impl<128, 128>(s, a, tmK, tmV, num_sms, stream);
     if (s.D == 64 && s.blk == 64) return launch_impl<64, 64>(s, a, tmK, tmV, num_sms, stream);
     if (s.D == 64 && s.blk == 128) return launch_impl<64, 128>(s, a, tmK, tmV, num_sms, stream);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_step(const Shape& s, const StepLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                               int num_sms, cudaStream_t stream) {
+#define SEER_STEP(D_, B_, G_) \
+    if (s.D == D_ && s.blk == B_ && s.dg == G_) return step_impl<D_, B_, G_>(s, a, tmK, tmV, num_sms, stream)
+    SEER_STEP(128, 64, 128);
+    SEER_STEP(128, 128, 128);
+    SEER_STEP(128, 64, 64);
+    SEER_STEP(128, 128, 64);
+    SEER_STEP(64, 64, 128);
+    SEER_STEP(64, 128, 128);
+    SEER_STEP(64, 64, 64);
+    SEER_STEP(64, 128, 64);
+#undef SEER_STEP
     return cudaErrorInvalidValue;
 }
 

@@ -44,6 +44,7 @@
 #ifndef SEER_H_
 #define SEER_H_
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -185,10 +186,68 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
                          int32_t num_splits, void* out, float* lse_out, cudaStream_t stream);
 
 /*
+ * The whole decode step, a1..a5, in ONE cooperative launch (one CTA per SM).
+ * Phase 1 spreads the (b, kvh) rows over the CTAs: refresh kpool for the
+ * blocks touching [upd_start[b], L_b) (NULL: the last block only, i.e. the
+ * token just appended), score every other block with the same arithmetic
+ * as seer_gate_scores, and select as seer_select_blocks does (bit-identical
+ * block lists). After a grid-wide barrier, phase 2 is seer_sparse_decode's
+ * schedule; the last CTA to finish a row merges its slots into out / lse_out
+ * as seer_combine does. One launch, no host synchronisation.
+ *
+ *   q, k_cache, v_cache, w_q, w_k, seq_lens   as above
+ *   upd_start     int32 [B] or NULL (NULL: L_b - 1)
+ *   budget_tokens a positive multiple of block_size; kmax = budget_tokens / block_size
+ *   sm_scale      <= 0 selects 1/sqrt(D)
+ *   kpool         fp32 [B, Hkv, NBmax, dg], read, and written for refreshed blocks
+ *   block_idx     int32 [B, Hkv, kmax] (output: the kept blocks, as seer_select_blocks)
+ *   num_selected  int32 [B, Hkv]       (output)
+ *   out           bf16 [B, Hq, D]      (output)
+ *   lse_out       fp32 [B, Hq]         (output, may be NULL)
+ *   workspace     device scratch of at least seer_decode_step_workspace_size()
+ *                 bytes, 256-byte aligned, ZERO-FILLED before its first use; every
+ *                 call leaves it ready for the next one (re-zero it after a call
+ *                 that reported a wait failure). Calls that share a workspace
+ *                 must not overlap on the GPU.
+ * Errors: as the separate calls; SEER_ERR_CUDA also when the cooperative launch
+ * cannot place one CTA on every SM (e.g. the device is shared with other work).
+ */
+seer_status seer_decode_step_workspace_size(const seer_dims* dims, int32_t budget_tokens, size_t* bytes);
+
+seer_status seer_decode_step(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                             const float* w_q, const float* w_k, const int32_t* seq_lens, const int32_t* upd_start,
+                             int32_t budget_tokens, float sm_scale, float* kpool, int32_t* block_idx,
+                             int32_t* num_selected, void* out, float* lse_out, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Slots per (b, h) that let seer_sparse_decode use every SM of the current
  * device: min(kmax, number of SMs). Host-only query (no launch).
  */
 seer_status seer_default_num_splits(int32_t kmax, int32_t* num_splits);
+
+/*
+ * Failure detection (no page counterpart). Every wait inside the decode kernel
+ * is bounded (1 s); a CTA that gives up writes NaN into the slot it was
+ * producing (so the combined output is NaN) and increments a device counter.
+ *
+ * seer_decode_wait_failures: *count = that counter for the current device
+ * (0 in normal operation); reset != 0 clears it. Synchronous: it waits for
+ * work already queued on the legacy default stream.
+ */
+seer_status seer_decode_wait_failures(uint32_t* count, int32_t reset);
+
+/*
+ * Self-test of the bounded wait: one CTA waits, for at most limit_ns
+ * (0 .. 2e9), on an mbarrier that nothing arrives at. *timed_out = 1 when the
+ * wait gave up as designed (0 if it completed, which would be a fault of the
+ * wait). The device stays usable afterwards. Synchronous (device-wide sync).
+ */
+seer_status seer_wait_selftest(int64_t limit_ns, int32_t* timed_out);
+
+/* The CUDA error behind the last SEER_ERR_CUDA returned on the calling host
+ * thread ("name: description"), or "no error". Valid until the next call. */
+const char* seer_last_error_string(void);
 
 /* A short static description of a status code. */
 const char* seer_status_string(seer_status status);

@@ -71,6 +71,8 @@ def check_scores(gpu_s, ora_s, lens, blk):
     worst = 0.0
     for b in range(len(lens)):
         nb = -(-int(lens[b]) // blk)
+        if nb == 0:
+            continue
         err = np.abs(gpu_s[b, :, :nb] - ora_s[b, :, :nb]).max()
         worst = max(worst, float(err))
     assert worst <= SCORE_ABS, f"gate score error {worst:.3e} > {SCORE_ABS}"
@@ -99,5 +101,6 @@ def check_attention(gpu_out, gpu_lse, ora_out, ora_lse):
     assert err.mean() <= OUT_MEAN_ABS, f"mean abs error {err.mean():.3e}"
     finite = np.isfinite(ora_lse)
     assert (np.isfinite(gpu_lse) == finite).all()
-    assert np.abs(gpu_lse[finite] - ora_lse[finite]).max() <= LSE_ABS
+    if finite.any():
+        assert np.abs(gpu_lse[finite] - ora_lse[finite]).max() <= LSE_ABS
     return float(err.max()), float(err.mean())

@@ -88,3 +88,28 @@ def test_python_wrapper_raises_on_error():
     with pytest.raises(api.SeerError) as e:
         api.seer_combine(_dims(head_dim=96), FAKE, FAKE, 4, FAKE, None, stream=0)
     assert e.value.status == api.SEER_ERR_UNSUPPORTED
+
+
+def test_failure_detection_entries_validate_on_host():
+    L = api.LIB
+    assert L.seer_decode_wait_failures(None, 0) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_wait_selftest(-1, ctypes.byref(ctypes.c_int32())) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_wait_selftest(3_000_000_000, ctypes.byref(ctypes.c_int32())) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_wait_selftest(1000, None) == api.SEER_ERR_INVALID_ARG
+
+
+def test_decode_step_validates_on_host():
+    d = _dims()
+    L = api.LIB
+    args = [FAKE] * 6
+    sz = ctypes.c_size_t(0)
+    assert L.seer_decode_step_workspace_size(ctypes.byref(d), 100, ctypes.byref(sz)) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_decode_step_workspace_size(ctypes.byref(d), 64, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_decode_step(ctypes.byref(_dims(head_dim=96)), *args, None, 64, 0.0, FAKE, FAKE, FAKE, FAKE, None,
+                              FAKE, 1 << 30, None) == api.SEER_ERR_UNSUPPORTED
+    assert L.seer_decode_step(ctypes.byref(d), *args, None, 64, 0.0, FAKE, FAKE, FAKE, FAKE, None, None, 1 << 30,
+                              None) == api.SEER_ERR_INVALID_ARG           # no workspace
+    assert L.seer_decode_step(ctypes.byref(d), *args, None, 100, 0.0, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30,
+                              None) == api.SEER_ERR_INVALID_ARG           # budget not a multiple of blk
+    assert L.seer_decode_step(ctypes.byref(d), *args, None, 64, 0.0, FAKE, FAKE, FAKE, FAKE, None, FAKE + 16,
+                              1 << 30, None) == api.SEER_ERR_INVALID_ARG  # workspace not 256-byte aligned

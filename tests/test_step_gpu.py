@@ -1,0 +1,107 @@
+"""The fused single-launch decode step (seer_decode_step) against the oracle
+and against the separate five-call path.
+
+* block lists: bit-exact with the oracle's (near-tie rows excluded) and
+  bit-identical with seer_select_blocks' (same arithmetic, gate_core.cuh);
+* refreshed pooled keys: identical to seer_kpool_update's;
+* output: within the attention tolerance of the fp64 oracle given the same
+  block list, and of the five-call path;
+* repeated calls on one workspace give identical results (the in-kernel
+  counters and the grid barrier reset themselves).
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_seer_b200 import api
+from block_sparse_attention_seer_b200 import workloads as W
+from oracle import oracle as O
+
+from gpu_helpers import check_attention, check_indices, oracle_bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_both(wl, inp):
+    """Separate five-call step and fused step from the same pooled cache."""
+    sep = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
+    sep.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
+    fus = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
+    fus.kpool.copy_(sep.kpool)
+    sep.set_update_start(inp["seq_lens"])
+    sep.step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+    fus.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+    torch.cuda.synchronize()
+    return sep, fus
+
+
+def check_step(wl, inp, batches=None):
+    sep, fus = run_both(wl, inp)
+    assert torch.equal(fus.block_idx, sep.block_idx)
+    assert torch.equal(fus.num_selected, sep.num_selected)
+    assert torch.equal(fus.kpool, sep.kpool)
+    a = fus.out.float().cpu().numpy()
+    b = sep.out.float().cpu().numpy()
+    assert np.abs(a - b).max() <= 1e-2
+    sel = slice(None) if batches is None else list(batches)
+    c = oracle_bits(inp, batches)
+    ora = O.step(c["q"], c["k"], c["v"], c["w_q"], c["w_k"], c["lens"], wl.block_size, wl.budget_tokens)
+    gidx = fus.block_idx.cpu().numpy()[sel]
+    gns = fus.num_selected.cpu().numpy()[sel]
+    excluded = check_indices(gidx, gns, ora["block_idx"], ora["num_selected"], ora["scores"], c["lens"],
+                             wl.block_size)
+    o, l = O.attend(c["q"], c["k"], c["v"], c["lens"], gidx, gns, wl.block_size)
+    mx, mean = check_attention(fus.out.cpu().double().numpy()[sel], fus.lse.cpu().double().numpy()[sel], o, l)
+    return fus, excluded, mx, mean
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_fused_tiny(seed):
+    wl = W.WORKLOADS["tiny"]
+    check_step(wl, to_dev(W.make_inputs(wl, seed=seed)))
+
+
+@pytest.mark.parametrize("shape", [
+    (3, 32, 8, 128, 128, 64, 4096, [4096, 3001, 1], 1024),
+    (2, 40, 8, 128, 128, 128, 8192, [8192, 5000], 1280),
+    (2, 8, 1, 64, 128, 128, 2048, [2000, 129], 512),
+    (4, 2, 2, 64, 64, 64, 1024, [64, 65, 127, 1000], 256),
+    (2, 4, 2, 128, 64, 64, 3000, [2999, 1500], 640),
+    (5, 8, 2, 128, 128, 64, 512, [0, 1, 64, 512, 300], 64),
+    (5, 8, 2, 128, 128, 64, 512, [0, 1, 64, 512, 300], 4096),
+])
+def test_fused_small_shapes(shape):
+    B, Hq, Hkv, D, dg, blk, Lmax, lens, budget = shape
+    wl = W.Workload("fused", B, Hq, Hkv, D, dg, blk, Lmax, budget)
+    check_step(wl, to_dev(W.make_inputs(wl, seed=12, pad_value=float("nan"), seq_lens=np.array(lens, np.int32))))
+
+
+def test_fused_repeated_calls_reuse_workspace():
+    wl = W.Workload("repeat", 3, 32, 8, 128, 128, 64, 4096, 1024)
+    inp = to_dev(W.make_inputs(wl, seed=13, seq_lens=np.array([4096, 3001, 77], np.int32)))
+    st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
+    st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
+    outs = []
+    for _ in range(4):
+        st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+        torch.cuda.synchronize()
+        outs.append((st.out.clone(), st.lse.clone(), st.block_idx.clone()))
+    for o, l, i in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1]) and torch.equal(i, outs[0][2])
+    ws = st.workspace()
+    assert int(ws[:4].view(torch.int32).item()) == 0          # grid barrier arrivals back at zero
+    assert api.seer_decode_wait_failures() == 0
+
+
+@pytest.mark.parametrize("name,batches", [
+    ("decode_b16", [0, 15]),
+    ("large_block", [3]),
+    ("ragged", [0, 63]),
+    ("sweep_b1_keep10", None),
+    ("sweep_b4_keep50", [2]),
+])
+def test_fused_full_size(name, batches):
+    wl = W.WORKLOADS[name]
+    inp = W.make_inputs(wl, seed=0, device="cuda", pad_value=float("nan") if wl.ragged else None)
+    _, excluded, mx, mean = check_step(wl, inp, batches)
+    print(f"fused {name}: near-tie rows excluded {excluded}, out max {mx:.2e} mean {mean:.2e}")
