@@ -51,6 +51,7 @@ def _load_library():
         "seer_decode_wait_failures": [P, I32],
         "seer_decode_step_workspace_size": [D, I32, P],
         "seer_decode_step": [D, P, P, P, P, P, P, P, I32, F32, P, P, P, P, P, P, ctypes.c_size_t, P],
+        "seer_decode_step_noalloc": [D, P, P, P, P, P, P, P, I32, F32, P, P, P, P, P, P],
         "seer_wait_selftest": [ctypes.c_int64, P],
     }
     for name, args in sig.items():
@@ -149,6 +150,15 @@ def seer_decode_step(dims, q, k_cache, v_cache, w_q, w_k, seq_lens, upd_start, b
         ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(w_q), _ptr(w_k), _ptr(seq_lens),
         _ptr(upd_start), int(budget_tokens), float(sm_scale), _ptr(kpool), _ptr(block_idx), _ptr(num_selected),
         _ptr(out), _ptr(lse_out), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def seer_decode_step_noalloc(dims, q, k_cache, v_cache, w_q, w_k, seq_lens, upd_start, budget_tokens, sm_scale,
+                             kpool, block_idx, num_selected, out, lse_out, stream=None):
+    """seer_decode_step with its scratch in the library's static device array (no workspace, no allocation)."""
+    _check("seer_decode_step_noalloc", LIB.seer_decode_step_noalloc(
+        ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(w_q), _ptr(w_k), _ptr(seq_lens),
+        _ptr(upd_start), int(budget_tokens), float(sm_scale), _ptr(kpool), _ptr(block_idx), _ptr(num_selected),
+        _ptr(out), _ptr(lse_out), _stream(stream)))
 
 
 def seer_default_num_splits(kmax: int) -> int:

@@ -233,6 +233,51 @@ seer_status seer_decode_step(const seer_dims* dims, const void* q, const void* k
     return from_cuda(seer::launch_decode_step(s, a, tmk, tmv, nsm, stream));
 }
 
+seer_status seer_decode_step_noalloc(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                                     const float* w_q, const float* w_k, const int32_t* seq_lens,
+                                     const int32_t* upd_start, int32_t budget_tokens, float sm_scale, float* kpool,
+                                     int32_t* block_idx, int32_t* num_selected, void* out, float* lse_out,
+                                     cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !k_cache || !v_cache || !w_q || !w_k || !seq_lens || !kpool || !block_idx || !num_selected || !out)
+        return SEER_ERR_INVALID_ARG;
+    if (budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(w_q, 16) ||
+        !aligned(w_k, 16) || !aligned(kpool, 16) || !aligned(out, 2))
+        return SEER_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
+    if (s.NBmax > 16384) return SEER_ERR_UNSUPPORTED;
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return SEER_ERR_CUDA;
+    if (seer::step_workspace_layout(s, budget_tokens / s.blk, nsm).total > seer::static_scratch_bytes()) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "seer_decode_step_noalloc: scratch for these sizes exceeds the %zu-byte static array; use "
+                 "seer_decode_step with a workspace", seer::static_scratch_bytes());
+        return SEER_ERR_UNSUPPORTED;
+    }
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, k_cache, s) || !encode_cache_map(&tmv, v_cache, s)) return SEER_ERR_CUDA;
+    seer::StepLaunch a;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.w_q = w_q;
+    a.w_k = w_k;
+    a.seq_lens = seq_lens;
+    a.upd_start = upd_start;
+    a.budget_tokens = budget_tokens;
+    a.sm_scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
+    a.kpool = kpool;
+    a.block_idx = block_idx;
+    a.num_selected = num_selected;
+    a.out = out;
+    a.lse_out = lse_out;
+    a.workspace = nullptr;
+    return from_cuda(seer::launch_decode_step_static(s, a, tmk, tmv, nsm, stream));
+}
+
 seer_status seer_default_num_splits(int32_t kmax, int32_t* num_splits) {
     if (kmax < 1 || !num_splits) return SEER_ERR_INVALID_ARG;
     const int nsm = device_sm_count();

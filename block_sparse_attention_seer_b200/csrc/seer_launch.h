@@ -69,6 +69,12 @@ WorkspaceLayout step_workspace_layout(const Shape& s, int kmax, int num_sms);
 cudaError_t launch_decode_step(const Shape& s, const StepLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                int num_sms, cudaStream_t stream);
 
+// The same step with its scratch in a static device array instead of a caller
+// workspace (no allocation anywhere); static_scratch_bytes() is the array's size.
+size_t static_scratch_bytes();
+cudaError_t launch_decode_step_static(const Shape& s, StepLaunch a, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                      int num_sms, cudaStream_t stream);
+
 // Failure detection: the decode kernel's count of CTAs that gave up on a
 // bounded wait, and a self-test of the bounded wait (synchronous).
 cudaError_t read_decode_wait_failures(unsigned int* count, bool reset);

@@ -929,6 +929,43 @@ cudaError_t launch_sparse_decode(const Shape& s, const DecodeLaunch& a, const CU
     return cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------- step without a caller workspace
+//
+// Some callers cannot allocate device memory for the step's scratch: a plugin
+// that its host framework hands nothing but input and output tensors, or a
+// decode loop that must not call cudaMalloc (it can synchronise the device)
+// once serving has started. For them the step's scratch lives in this
+// file-scope array, one copy on every GPU that loads the library, held until
+// the process exits. Its address is looked up once per device.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+size_t static_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t launch_decode_step_static(const Shape& s, StepLaunch a, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                      int num_sms, cudaStream_t stream) {
+    constexpr int kMaxDevices = 64;
+    static void* scratch[kMaxDevices] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (!scratch[dev]) {  // set-up, once per device, with that device current
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        scratch[dev] = ptr;
+    }
+    const WorkspaceLayout wl = step_workspace_layout(s, a.budget_tokens / s.blk, num_sms);
+    if (wl.total > kStaticScratchBytes) return cudaErrorInvalidValue;
+    // The array keeps the previous call's contents: the barrier words and row
+    // counts must start at zero.
+    e = cudaMemsetAsync(scratch[dev], 0, wl.o_part, stream);
+    if (e != cudaSuccess) return e;
+    a.workspace = scratch[dev];
+    return launch_decode_step(s, a, tmK, tmV, num_sms, stream);
+}
+
 cudaError_t launch_decode_step(const Shape& s, const StepLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                int num_sms, cudaStream_t stream) {
 #define SEER_STEP(D_, B_, G_) \

@@ -221,6 +221,32 @@ seer_status seer_decode_step(const seer_dims* dims, const void* q, const void* k
                              size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * seer_decode_step without a workspace argument, for callers that cannot
+ * allocate device memory: e.g. a plugin whose host framework passes it only
+ * its input and output tensors, or a serving loop that may not call
+ * cudaMalloc (which can synchronise the whole device) once it is running.
+ * (No counterpart in the papers: an interface convenience.)
+ *
+ * The scratch lives in a static device array of 32 MiB inside the library:
+ * every GPU that loads the library holds one copy until the process exits.
+ * Sizes whose scratch (seer_decode_step_workspace_size) exceeds 32 MiB are
+ * rejected with SEER_ERR_UNSUPPORTED (seer_last_error_string says why); use
+ * seer_decode_step for them. Nothing is allocated or freed: the first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current, so make that first call before any stream
+ * capture; each call then clears the array's counters (an async memset on
+ * `stream`) and launches the same kernel as seer_decode_step.
+ * Every call on a device shares the one array: calls whose executions
+ * overlap on the GPU (different streams, no ordering between them) race.
+ * Arguments, outputs and errors otherwise as seer_decode_step.
+ */
+seer_status seer_decode_step_noalloc(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                                     const float* w_q, const float* w_k, const int32_t* seq_lens,
+                                     const int32_t* upd_start, int32_t budget_tokens, float sm_scale, float* kpool,
+                                     int32_t* block_idx, int32_t* num_selected, void* out, float* lse_out,
+                                     cudaStream_t stream);
+
+/*
  * Slots per (b, h) that let seer_sparse_decode use every SM of the current
  * device: min(kmax, number of SMs). Host-only query (no launch).
  */
