@@ -13,8 +13,8 @@
 // scan over kpool is the HBM cost. A thread-block cluster of C CTAs serves one
 // row: each CTA projects dg/C components of W_q qbar, the cluster exchanges
 // them through distributed shared memory, and each CTA then scores its own
-// contiguous chunk of the row's blocks, one warp per block row of kpool
-// (16-byte loads, shuffle reduction).
+// contiguous chunk of the row's blocks, one lane quad per block row
+// (quad_row_dot, the same summation order as the fused step).
 #include <cooperative_groups.h>
 
 #include "gate_core.cuh"
@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kThreads)
                        float* __restrict__ scores, int Hq, int Hkv, int G, int blk, int Lmax, int NBmax) {
     __shared__ float qbar[D];
     __shared__ float qg_part[DG];  // components this CTA projects (others stay unused)
-    __shared__ float qg[DG];
+    __shared__ __align__(16) float qg[DG];
 
     cg::cluster_group cluster = cg::this_cluster();
     const int csize = (int)cluster.num_blocks();
@@ -67,31 +67,15 @@ __global__ void __launch_bounds__(kThreads)
     const int per = (NB + csize - 1) / csize;
     const int j0 = crank * per;
     const int j1 = min(NB, j0 + per);
-    constexpr int kVecG = DG / 32;
-    float gv[kVecG];
+    // one lane quad per block row, 8 consecutive rows per warp step
     const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
-#pragma unroll
-    for (int u = 0; u < kVecG; ++u) gv[u] = qg[lane * kVecG + u];
-    using Vec = GateVec<DG>;
-    const Vec* kp = reinterpret_cast<const Vec*>(kpool + (size_t)row * NBmax * DG) + lane;
+    const float* kp = kpool + (size_t)row * NBmax * DG;
     float* out = scores + (size_t)row * NBmax;
-    constexpr int kUnroll = 8;
-    for (int jb = j0 + warp * kUnroll; jb < j1; jb += kWarps * kUnroll) {
-        Vec v[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int j = min(jb + u, j1 - 1);  // clamped duplicate loads past j1 are never stored
-            v[u] = __ldcs(kp + (size_t)j * (DG / kVecG));
-        }
-        float d[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) d[u] = gate_dot<DG>(v[u], gv);
-        if (lane < kUnroll && jb + lane < j1) {
-            float x = d[0];
-#pragma unroll
-            for (int u = 1; u < kUnroll; ++u) x = (lane == u) ? d[u] : x;
-            out[jb + lane] = x * inv_sqrt_dg;
-        }
+    const int quad = lane >> 2, qlane = lane & 3;
+    for (int jb = j0 + warp * 8; jb < j1; jb += kWarps * 8) {
+        const int j = min(jb + quad, j1 - 1);  // lanes past j1 repeat the last row and store nothing
+        const float d = quad_row_dot<DG>(kp + (size_t)j * DG, j, qg, qlane);
+        if (qlane == 0 && jb + quad < j1) out[j] = d * inv_sqrt_dg;
     }
 }
 

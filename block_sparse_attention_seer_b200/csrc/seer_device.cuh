@@ -159,6 +159,13 @@ __device__ __forceinline__ float warp_max(float v) {
 // warp per row with 8 rows in flight: each lane holds D/32 entries of v
 // (vd) and reads the matching 16- or 8-byte piece of each W row (coalesced
 // across the warp). Lane 0 of the warp returns the dot through `sink`.
+// One lane's piece of a W-row . v dot (4 or 2 columns); every matvec of the
+// library goes through these, so equal inputs give equal bits.
+__device__ __forceinline__ float piece_dot(const float4& w, const float* v) {
+    return w.x * v[0] + w.y * v[1] + w.z * v[2] + w.w * v[3];
+}
+__device__ __forceinline__ float piece_dot(const float2& w, const float* v) { return w.x * v[0] + w.y * v[1]; }
+
 template <int D, typename Sink>
 __device__ __forceinline__ void warp_matvec_rows(const float* __restrict__ W, const float (&vd)[D / 32], int first,
                                                  int end, int stride, Sink sink) {
@@ -172,13 +179,8 @@ __device__ __forceinline__ void warp_matvec_rows(const float* __restrict__ W, co
             d[u] = 0.f;
             if (e < end) {
                 const float* we = W + (size_t)e * D + lane * kVec;
-                if constexpr (kVec == 4) {
-                    const float4 w = *reinterpret_cast<const float4*>(we);
-                    d[u] = w.x * vd[0] + w.y * vd[1] + w.z * vd[2] + w.w * vd[3];
-                } else {
-                    const float2 w = *reinterpret_cast<const float2*>(we);
-                    d[u] = w.x * vd[0] + w.y * vd[1];
-                }
+                if constexpr (kVec == 4) d[u] = piece_dot(*reinterpret_cast<const float4*>(we), vd);
+                else d[u] = piece_dot(*reinterpret_cast<const float2*>(we), vd);
             }
         }
 #pragma unroll
@@ -190,6 +192,15 @@ __device__ __forceinline__ void warp_matvec_rows(const float* __restrict__ W, co
             if (lane == 0 && e < end) sink(e, x);
         }
     }
+}
+
+// atomicAdd with acquire-release semantics at GPU scope: publishes every write
+// this thread has observed (e.g. its CTA's writes before a __syncthreads) and
+// sees every write published by earlier adds to the same counter.
+__device__ __forceinline__ unsigned int atomic_add_acq_rel(unsigned int* p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 
 // Named barrier over `threads` threads (a multiple of 32), id 1..15.

@@ -62,7 +62,7 @@ struct StepLaunch {
 
 // Byte offsets inside the step's workspace.
 struct WorkspaceLayout {
-    size_t grid_bar, row_done, o_part, lse_part, total;
+    size_t grid_bar, row_done, row_cnt, qg_flag, counters_end, qg, keys, o_part, lse_part, total;
 };
 WorkspaceLayout step_workspace_layout(const Shape& s, int kmax, int num_sms);
 

@@ -6,19 +6,17 @@
 // highest-scoring blocks among 0 .. NB_b - 2 (k_b = min(budget/blk, NB_b)),
 // equal scores going to the lower index, written in ascending order.
 //
-// One CTA per row. Scores become order-preserving 32-bit keys in shared
-// memory; an MSB-first radix select (4 passes of 8 bits, warp-aggregated
-// shared-memory histograms) finds the threshold key tau of the (k_b-1)-th
-// largest score and how many keys equal to tau are needed. A block-wide scan
-// in index order then ranks the tau-ties (lowest indices win) and compacts
-// the kept indices, which come out ascending by construction.
+// One CTA per row (select_row, gate_core.cuh). Scores become
+// order-preserving 32-bit keys in shared memory; a radix select from the top
+// (12-bit histogram, then an exact warp sort of the boundary bucket) finds the
+// kept set, and a scan in index order writes it, ascending by construction.
 #include "gate_core.cuh"
 #include "seer_launch.h"
 
 namespace seer {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 
 __global__ void __launch_bounds__(kThreads)
     select_blocks_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int Hkv, int Lmax,
@@ -41,11 +39,11 @@ __global__ void __launch_bounds__(kThreads)
 cudaError_t launch_select_blocks(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax,
                                  int32_t* block_idx, int32_t* num_selected, cudaStream_t stream) {
     const size_t smem = (size_t)s.NBmax * sizeof(uint32_t);
-    if (smem > 48 * 1024) {
+    if (smem > 16 * 1024) {  // above what is left beside the static histogram
         static bool attr_done = false;
         if (!attr_done) {
             cudaError_t e = cudaFuncSetAttribute(select_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 64 * 1024 + 1024);
+                                                 16384 * 4);
             if (e != cudaSuccess) return e;
             attr_done = true;
         }

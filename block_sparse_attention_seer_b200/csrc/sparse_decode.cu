@@ -59,7 +59,10 @@ namespace {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kThreads = kConsumerThreads + 32;       // standalone decode: consumers + producer
+constexpr int kHelperWarp0 = kConsumerWarps + 1;       // fused step: + 3 helper warps
+constexpr int kHelperThreads = 96;
+constexpr int kStepThreads = kThreads + kHelperThreads;  // 12 warps: the register budget of 9 (allocated as 12)
 constexpr int kMaxStages = 8;
 constexpr int kMaxGateStages = 8;
 constexpr int kSmemLimit = 232448;       // 227 KB of opt-in dynamic shared memory per CTA
@@ -104,9 +107,14 @@ struct StepParams {
     __nv_bfloat16* out;
     float* lse_out;
     unsigned int* grid_bar;  // {arrivals, generation}
-    unsigned int* row_done;  // [rows] finished slots per row
-    int rows, NBmax;
+    unsigned int* row_done;  // [rows] finished decode slots per row
+    unsigned int* row_cnt;   // [rows] finished phase-1 pieces per row
+    unsigned int* qg_flag;   // [rows] the row's projected query is in qg_g
+    float* qg_g;             // [rows, dg] projected queries, written by each row's first CTA
+    uint32_t* keys_g;        // [rows, NBmax] order keys of the block scores
+    int rows, NBmax, dg;
     int keys_off, chunk_off, n_gate_stages;  // phase-1 layout inside the stage ring
+    int refresh_off;                         // phase-2 pool scratch (outside the ring)
 };
 
 // Shared-memory info words after the per-stage `valid` counts.
@@ -174,6 +182,7 @@ struct Smem {
     __device__ __forceinline__ uint32_t empty(int st) const { return bars + 8u * (nst + st); }
     __device__ __forceinline__ uint32_t cons() const { return bars + 16u * nst; }
     __device__ __forceinline__ uint32_t gate(int st) const { return bars + 16u * nst + 8u + 8u * st; }
+    __device__ __forceinline__ uint32_t helper() const { return bars + 16u * nst + 8u + 8u * kMaxGateStages; }
 };
 
 __device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) {
@@ -191,6 +200,7 @@ __device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) 
         }
         mbar_init(m.cons(), kConsumerThreads);
         for (int st = 0; st < kMaxGateStages; ++st) mbar_init(m.gate(st), 1);
+        mbar_init(m.helper(), kHelperThreads);
         for (int i = 0; i < kInfoWords; ++i) m.info[i] = 0;
         fence_mbar_init();
     }
@@ -289,15 +299,13 @@ template <int D>
 __device__ void merge_row_if_last(const Params& p, const StepParams& f, const Smem& m, const Segment& s,
                                   uint32_t& cph) {
     const int ctid = threadIdx.x;
-    __threadfence();  // this CTA's slot writes before its count
-    if (!consumer_sync(m, cph)) return;
+    if (!consumer_sync(m, cph)) return;  // the CTA's slot writes, then its release-add
     if (ctid == 0) {
-        const unsigned int done = atomicAdd(f.row_done + s.row, 1u) + 1u;
+        const unsigned int done = atomic_add_acq_rel(f.row_done + s.row, 1u) + 1u;
         m.info[kInfoMergeRow] = (done == (unsigned int)s.nslots);
     }
-    if (!consumer_sync(m, cph)) return;
+    if (!consumer_sync(m, cph)) return;  // the acquire, then every consumer reads the slots
     if (!m.info[kInfoMergeRow]) return;
-    __threadfence();  // other CTAs' slots, published before their counts
     const size_t head0 = (size_t)s.b * p.Hq + (size_t)s.kvh * p.G;
     const int ns = s.nslots;
     float* w = m.merge;  // [G][ns] normalised slot weights (the merge area is free here)
@@ -545,6 +553,49 @@ __device__ void decode_consumers(const Params& p, const StepParams& f, const Sme
     }
 }
 
+// ---------------------------------------------------------------- fused step: helper warps
+
+// First block to refresh for sequence b (upd_start, by default the token just appended).
+__device__ __forceinline__ int refresh_start_block(const StepParams& f, int b, int L, int NB, int blk) {
+    int st0 = f.upd_start ? f.upd_start[b] : L - 1;
+    st0 = st0 < 0 ? 0 : st0;
+    return min(st0 / blk, NB);
+}
+
+// Phase 2, warps 9..11, beside the decode: refresh the pooled key of the open
+// last block of every row whose first slot this CTA holds. Phase 1 never reads
+// it (the last block is always kept), so it runs while the decode streams.
+template <int D, int BLK>
+__device__ void decode_helpers(const Params& p, const StepParams& f, const Smem& m, long long g0, long long g1) {
+    PoolSmem<D>& psm = *reinterpret_cast<PoolSmem<D>*>(m.base + f.refresh_off);
+    const int hwarp = ((int)threadIdx.x >> 5) - kHelperWarp0, lane = threadIdx.x & 31;
+    uint32_t hph = 0;
+    bool ok = true;
+    auto hsync = [&]() {
+        if (!ok) return;
+        mbar_arrive(m.helper());
+        ok = mbar_wait(m.helper(), hph);
+        hph ^= 1u;
+        if (!ok) record_failure(m.info);
+    };
+    for (int r = (int)(g0 / p.kmax); ok && (long long)r * p.kmax < g1; ++r) {
+        const Segment s = make_segment<true>(p, r, g0, g1);
+        if (s.slot != 0 || s.L == 0) continue;
+        const int NB = (s.L + BLK - 1) / BLK;
+        if (refresh_start_block(f, s.b, s.L, NB, BLK) > NB - 1) continue;
+        const int j = NB - 1;
+        pool_block_mean<D, BLK>(f.k_cache + ((size_t)r * p.Lmax + (size_t)j * BLK) * D, s.L - j * BLK, psm, hsync,
+                                kHelperWarp0 * 32);
+        float pv[D / 32];
+#pragma unroll
+        for (int u = 0; u < D / 32; ++u) pv[u] = psm.pooled[lane * (D / 32) + u];
+        float* dst = f.kpool + ((size_t)r * f.NBmax + j) * f.dg;
+        const float* W = f.w_k + (size_t)s.kvh * f.dg * D;
+        warp_matvec_rows<D>(W, pv, hwarp, f.dg, kHelperThreads / 32, [&](int e, float x) { dst[e] = x; });
+        hsync();  // the pool scratch is reused by the next row
+    }
+}
+
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registers as 12: <= 168 each
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -559,108 +610,289 @@ __global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registe
 
 // ---------------------------------------------------------------- fused step: phase 1 (gate + select)
 
+// One row of the rows a CTA meets in its phase-1 range.
+struct GateRow {
+    int r, b, kvh, L, NB, js;  // js: first block whose pooled key is refreshed
+    int s0, s1;                // cached positions [s0, s1) this CTA scores
+    int scored;                // the row's choice needs scores
+    int refresh_now;           // this CTA refreshes the competing blocks [js, NB-1) here
+};
+constexpr int kMaxBatchRows = 8;
+
 template <int D, int DG>
 struct GateScratch {
-    PoolSmem<D> pool;
-    SelectSmem<kThreads> sel;
-    alignas(16) float qbar[D];
-    alignas(16) float qg[DG];
+    alignas(16) float qbar[kMaxBatchRows][D];
+    alignas(16) float qg[kMaxBatchRows][DG];
     alignas(16) float kp_new[DG];
+    PoolSmem<D> pool;
+    GateRow rows[kMaxBatchRows];
+    int last_of[kMaxBatchRows];
 };
 static_assert(sizeof(GateScratch<128, 128>) <= kGateScratchBytes, "phase-1 scratch");
+static_assert(sizeof(SelectSmem<kStepThreads>) <= kGateChunkBytes, "the select scratch reuses a chunk stage");
+static_assert(sizeof(GateScratch<64, 128>) <= kGateScratchBytes, "phase-1 scratch");
 
+// Phase 1. The R x NBmax pooled-key positions (row-major, the layout of
+// kpool) are cut into gridDim.x equal contiguous ranges. Each CTA streams the
+// cached rows of its range into the stage ring (bulk copies), scores them
+// against the projected query of their row (a lane quad per row), and writes
+// order keys to the workspace. A per-row count of finished ranges tells the
+// last CTA of a row to run that row's selection. The open last block is never
+// a candidate, so its pooled key is refreshed in phase 2; only blocks that
+// compete (a refresh point before the last block) are refreshed here.
 template <int D, int BLK, int DG>
 __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) {
+    constexpr int kThreads = kStepThreads;
     constexpr int kWarps = kThreads / 32;
-    constexpr int kVecG = DG / 32;
     constexpr int kChunkRows = kGateChunkBytes / (DG * 4);
-    using Vec = GateVec<DG>;
+    constexpr int kVecD = D / 32;
+    using WVec = typename std::conditional<kVecD == 4, float4, float2>::type;
     GateScratch<D, DG>& sm = *reinterpret_cast<GateScratch<D, DG>*>(m.base);
     uint32_t* keys = reinterpret_cast<uint32_t*>(m.base + f.keys_off);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = lane >> 2, qlane = lane & 3;
     const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
-    int chunk_it = 0;  // bulk-copy stages used so far (same count on every thread)
+    const long long V1 = (long long)f.rows * f.NBmax;
+    // With no more rows than CTAs every CTA takes one whole row (no hand-offs:
+    // its keys stay in shared memory and it selects right after scoring);
+    // otherwise the positions are spread over every CTA.
+    const int G1 = f.rows <= (int)gridDim.x ? f.rows : (int)gridDim.x;
+    if ((int)blockIdx.x >= G1) return;
+    const long long h0 = (long long)blockIdx.x * V1 / G1;
+    const long long h1 = (long long)(blockIdx.x + 1) * V1 / G1;
+    const bool whole_rows = G1 == f.rows;
+    // Rows r with r * NBmax < h1, from the row holding h0: exactly the rows
+    // whose [first, last] covering-CTA interval contains this CTA (an empty
+    // range strictly inside a row still counts for that row).
+    const int r_stop = (int)((h1 + f.NBmax - 1) / f.NBmax);
+    int chunk_it = 0;  // bulk copies consumed so far (the same count on every thread)
 
-    for (int r = blockIdx.x; r < f.rows; r += gridDim.x) {
-        const int b = r / p.Hkv, kvh = r - b * p.Hkv;
-        const int L = clamp_len(p.seq_lens[b], p.Lmax);
-        const int NB = (L + BLK - 1) / BLK;
-        const int kb = p.kmax < NB ? p.kmax : NB;
-        int js = NB;  // first block whose pooled key is refreshed
-        if (NB > 0) {
-            int st0 = f.upd_start ? f.upd_start[b] : L - 1;
-            st0 = st0 < 0 ? 0 : st0;
-            js = min(st0 / BLK, NB);
-        }
-        const int ncand = NB - 1;
-        const bool scored = kb - 1 > 0 && kb - 1 < ncand;  // otherwise the choice needs no score
-        const int nscan = scored ? min(js, ncand) : 0;      // cached rows to score
-        const int nchunks = (nscan + kChunkRows - 1) / kChunkRows;
-        float* kp_row = f.kpool + (size_t)r * f.NBmax * DG;
-        auto chunk_dst = [&](int stage) { return m.sbase + (uint32_t)(f.chunk_off + stage * kGateChunkBytes); };
-        auto issue = [&](int i) {  // chunk i of this row into stage (chunk_it + i) % n
-            const int stage = (chunk_it + i) % f.n_gate_stages;
-            const int rows_i = min(kChunkRows, nscan - i * kChunkRows);
-            const uint32_t bytes = (uint32_t)(rows_i * DG * 4);
-            mbar_arrive_expect_tx(m.gate(stage), bytes);
-            bulk_load(chunk_dst(stage), kp_row + (size_t)i * kChunkRows * DG, bytes, m.gate(stage));
+    for (int r = (int)(h0 / f.NBmax); r < r_stop;) {
+        const int nb = min(kMaxBatchRows, r_stop - r);
+        // ---- (1) before anything else reaches DRAM: the projection weights of the
+        //      batch rows (first kQBatch outputs per warp), their lengths and
+        //      group-mean queries -- all independent loads, issued together
+        constexpr int kQBatch = 16;
+        // A row's first position lies in exactly one CTA's range: that CTA owns
+        // the row and projects its query; the owned rows of a batch are contiguous.
+        auto owner_of = [&](int row) {
+            const long long x = (long long)row * f.NBmax;
+            return x >= h0 && x < h1;
         };
-        if (tid == 0)
-            for (int i = 0; i < min(f.n_gate_stages, nchunks); ++i) issue(i);
-        // projected query of the group
-        group_query_mean<D>(p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G) * D, p.G, sm.qbar);
-        __syncthreads();
-        {
-            float qv[D / 32];
-#pragma unroll
-            for (int u = 0; u < D / 32; ++u) qv[u] = sm.qbar[lane * (D / 32) + u];
-            warp_matvec_rows<D>(f.w_q + (size_t)kvh * DG * D, qv, warp, DG, kWarps,
-                                [&](int e, float x) { sm.qg[e] = x; });
-        }
-        __syncthreads();
-        float gv[kVecG];
-#pragma unroll
-        for (int u = 0; u < kVecG; ++u) gv[u] = sm.qg[lane * kVecG + u];
-        // refresh the pooled keys of the open block(s); score them if they compete
-        const __nv_bfloat16* krow = f.k_cache + (size_t)r * p.Lmax * D;
-        for (int j = js; j < NB; ++j) {
-            pool_block_mean<D, BLK>(krow + (size_t)j * BLK * D, min(BLK, L - j * BLK), sm.pool);
-            float pv[D / 32];
-#pragma unroll
-            for (int u = 0; u < D / 32; ++u) pv[u] = sm.pool.pooled[lane * (D / 32) + u];
-            warp_matvec_rows<D>(f.w_k + (size_t)kvh * DG * D, pv, warp, DG, kWarps, [&](int e, float x) {
-                kp_row[(size_t)j * DG + e] = x;
-                sm.kp_new[e] = x;
-            });
-            __syncthreads();
-            if (scored && j < ncand && warp == 0) {
-                const float d = gate_dot<DG>(reinterpret_cast<const Vec*>(sm.kp_new)[lane], gv);
-                if (lane == 0) keys[j] = order_key(d * inv_sqrt_dg);
+        int own_first = nb, own_rows = 0;
+        for (int k = 0; k < nb; ++k)
+            if (owner_of(r + k)) {
+                own_first = min(own_first, k);
+                ++own_rows;
             }
-            __syncthreads();
+        const int total_q = own_rows * DG;  // outputs ordered by owned row, then e
+        auto owned_row = [&](int o) { return own_first + o / DG; };
+        WVec w[kQBatch];
+        if (total_q > 0) {
+#pragma unroll
+            for (int u = 0; u < kQBatch; ++u) {
+                const int o = min(warp + u * kWarps, total_q - 1);
+                const int k = owned_row(o), e = o % DG;
+                const int kvh = (r + k) % p.Hkv;
+                w[u] = *reinterpret_cast<const WVec*>(f.w_q + ((size_t)kvh * DG + e) * D + lane * kVecD);
+            }
         }
-        // score the cached rows as their chunks land
-        for (int i = 0; i < nchunks; ++i) {
+        if (tid < nb) {
+            GateRow& g = sm.rows[tid];
+            g.r = r + tid;
+            g.b = g.r / p.Hkv;
+            g.kvh = g.r - g.b * p.Hkv;
+            g.L = clamp_len(p.seq_lens[g.b], p.Lmax);
+            g.NB = (g.L + BLK - 1) / BLK;
+            g.js = g.NB > 0 ? refresh_start_block(f, g.b, g.L, g.NB, BLK) : g.NB;
+        }
+        for (int idx = tid; idx < nb * D; idx += kThreads) {
+            const int k = idx / D, d = idx - k * D;
+            const int row = r + k, b = row / p.Hkv, kvh = row - b * p.Hkv;
+            if (owner_of(row))
+                sm.qbar[k][d] = group_query_mean_at(p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G) * D, p.G, D, d);
+        }
+        __syncthreads();
+        if (tid < nb) {
+            GateRow& g = sm.rows[tid];
+            const long long rs = (long long)g.r * f.NBmax;
+            const int i0 = (int)(h0 > rs ? h0 - rs : 0);
+            const int i1 = (int)((h1 - rs) < f.NBmax ? (h1 - rs) : f.NBmax);
+            const int kb = p.kmax < g.NB ? p.kmax : g.NB;
+            const int ncand = g.NB - 1;
+            g.scored = kb - 1 > 0 && kb - 1 < ncand;
+            const int lim = g.scored ? min(g.js, ncand) : 0;
+            g.s0 = min(i0, lim);
+            g.s1 = min(i1, lim);
+            g.refresh_now = g.js < ncand && g.js >= i0 && g.js < i1;
+        }
+        __syncthreads();
+        auto nchunks_of = [&](int k) { return (sm.rows[k].s1 - sm.rows[k].s0 + kChunkRows - 1) / kChunkRows; };
+        int total_chunks = 0;
+        for (int k = 0; k < nb; ++k) total_chunks += nchunks_of(k);
+        auto chunk = [&](int i, int& k, int& j0, int& n) {
+            for (k = 0; k < nb - 1; ++k) {
+                const int c = nchunks_of(k);
+                if (i < c) break;
+                i -= c;
+            }
+            j0 = sm.rows[k].s0 + i * kChunkRows;
+            n = min(kChunkRows, sm.rows[k].s1 - j0);
+        };
+        auto issue = [&](int i) {
+            int k, j0, n;
+            chunk(i, k, j0, n);
+            const int stage = (chunk_it + i) % f.n_gate_stages;
+            const uint32_t bytes = (uint32_t)(n * DG * 4);
+            mbar_arrive_expect_tx(m.gate(stage), bytes);
+            bulk_load(m.sbase + (uint32_t)(f.chunk_off + stage * kGateChunkBytes),
+                      f.kpool + ((size_t)sm.rows[k].r * f.NBmax + j0) * DG, bytes, m.gate(stage));
+        };
+        // ---- (2) stream the cached pooled keys; meanwhile project the owned rows' queries
+        if (tid == 0)
+            for (int i = 0; i < min(f.n_gate_stages, total_chunks); ++i) issue(i);
+        if (total_q > 0) {
+#pragma unroll
+            for (int u = 0; u < kQBatch; ++u) {
+                const int o = warp + u * kWarps;
+                const int oc = min(o, total_q - 1);
+                const int k = owned_row(oc), e = oc % DG;
+                const float x = warp_sum(piece_dot(w[u], &sm.qbar[k][lane * kVecD]));
+                if (lane == 0 && o < total_q) sm.qg[k][e] = x;
+            }
+            for (int o0 = warp + kQBatch * kWarps; o0 < total_q; o0 += 8 * kWarps) {  // batches beyond the first
+                WVec w2[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int o = min(o0 + u * kWarps, total_q - 1);
+                    const int k = owned_row(o), e = o % DG;
+                    w2[u] = *reinterpret_cast<const WVec*>(f.w_q + ((size_t)sm.rows[k].kvh * DG + e) * D + lane * kVecD);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int o = o0 + u * kWarps;
+                    const int oc = min(o, total_q - 1);
+                    const int k = owned_row(oc), e = oc % DG;
+                    const float x = warp_sum(piece_dot(w2[u], &sm.qbar[k][lane * kVecD]));
+                    if (lane == 0 && o < total_q) sm.qg[k][e] = x;
+                }
+            }
+        }
+        __syncthreads();
+        // publish every owned projection first, then fetch the others' (their owners are
+        // lower-indexed CTAs that publish before they wait on anyone: no chains)
+        if (!whole_rows) {
+            for (int k = 0; k < nb; ++k)
+                if (owner_of(sm.rows[k].r) && sm.rows[k].scored)
+                    for (int e = tid; e < DG; e += kThreads) f.qg_g[(size_t)sm.rows[k].r * DG + e] = sm.qg[k][e];
+            __syncthreads();
+            if (tid < nb && owner_of(sm.rows[tid].r) && sm.rows[tid].scored)
+                asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(f.qg_flag + sm.rows[tid].r), "r"(1u) : "memory");
+        }
+        for (int k = 0; k < nb; ++k) {
+            const GateRow& g = sm.rows[k];
+            const bool needed = g.scored && (g.s1 > g.s0 || g.refresh_now);
+            if (!owner_of(g.r) && needed) {
+                if (tid == 0) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (true) {
+                        unsigned int v;
+                        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(f.qg_flag + g.r) : "memory");
+                        if (v) break;
+                        if (global_timer_ns() - t0 > kWaitLimitNs) {
+                            record_failure(m.info);
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                }
+                __syncthreads();
+                for (int e = tid; e < DG; e += kThreads) sm.qg[k][e] = __ldcg(f.qg_g + (size_t)g.r * DG + e);
+            }
+        }
+        __syncthreads();
+
+        // ---- (3) refresh and score competing blocks of a refresh point inside the range (multi-token appends)
+        for (int k = 0; k < nb; ++k) {
+            const GateRow& g = sm.rows[k];
+            if (!g.refresh_now) continue;
+            const __nv_bfloat16* krow = f.k_cache + (size_t)g.r * p.Lmax * D;
+            float* kp_row = f.kpool + (size_t)g.r * f.NBmax * DG;
+            for (int j = g.js; j < g.NB - 1; ++j) {
+                pool_block_mean<D, BLK>(krow + (size_t)j * BLK * D, min(BLK, g.L - j * BLK), sm.pool);
+                float pv[kVecD];
+#pragma unroll
+                for (int u = 0; u < kVecD; ++u) pv[u] = sm.pool.pooled[lane * kVecD + u];
+                warp_matvec_rows<D>(f.w_k + (size_t)g.kvh * DG * D, pv, warp, DG, kWarps, [&](int e, float x) {
+                    kp_row[(size_t)j * DG + e] = x;
+                    sm.kp_new[e] = x;
+                });
+                __syncthreads();
+                if (warp == 0) {
+                    const float d = quad_row_dot<DG>(sm.kp_new, j, sm.qg[k], qlane);
+                    if (lane == 0)
+                        (whole_rows ? keys : f.keys_g + (size_t)g.r * f.NBmax)[j] = order_key(d * inv_sqrt_dg);
+                }
+                __syncthreads();
+            }
+        }
+
+        // ---- (4) score the cached rows as their copies land (a lane quad per row)
+        for (int i = 0; i < total_chunks; ++i) {
+            int k, j0, n;
+            chunk(i, k, j0, n);
             const int stage = (chunk_it + i) % f.n_gate_stages;
             const uint32_t par = (uint32_t)(((chunk_it + i) / f.n_gate_stages) & 1);
             if (!mbar_wait(m.gate(stage), par)) record_failure(m.info);
-            const Vec* rows_v = reinterpret_cast<const Vec*>(m.base + f.chunk_off + stage * kGateChunkBytes) + lane;
-            const int j0 = i * kChunkRows;
-            const int nrows = min(kChunkRows, nscan - j0);
-            for (int jr = warp; jr < nrows; jr += kWarps) {
-                const float d = gate_dot<DG>(rows_v[(size_t)jr * 32], gv);
-                if (lane == 0) keys[j0 + jr] = order_key(d * inv_sqrt_dg);
+            const float* tile = reinterpret_cast<const float*>(m.base + f.chunk_off + stage * kGateChunkBytes);
+            uint32_t* kout = whole_rows ? keys : f.keys_g + (size_t)sm.rows[k].r * f.NBmax;
+            const float* qg = sm.qg[k];
+            for (int t0 = warp * 8; t0 < n; t0 += kWarps * 8) {
+                const int t = min(t0 + quad, n - 1);
+                const float d = quad_row_dot<DG>(tile + (size_t)t * DG, j0 + t, qg, qlane);
+                if (qlane == 0 && t0 + quad < n) kout[j0 + t] = order_key(d * inv_sqrt_dg);
             }
             fence_proxy_async_smem();  // these generic reads of the stage precede its next bulk copy
             __syncthreads();
-            if (tid == 0 && i + f.n_gate_stages < nchunks) issue(i + f.n_gate_stages);
+            if (tid == 0 && i + f.n_gate_stages < total_chunks) issue(i + f.n_gate_stages);
         }
-        chunk_it += nchunks;
+        chunk_it += total_chunks;
+
+        // ---- (5) count this CTA's pieces (one release-add per row, together);
+        //      the last CTA of a row selects its blocks
+        __syncthreads();  // every key of the batch written before the adds
+        if (tid < nb) {
+            const GateRow& g = sm.rows[tid];
+            const long long rs = (long long)g.r * f.NBmax;
+            if (whole_rows) {
+                sm.last_of[tid] = 1;  // the only CTA of its row
+            } else {
+                const int cf = (int)(((rs + 1) * G1 - 1) / V1);
+                const int cl = (int)(((rs + f.NBmax) * G1 - 1) / V1);
+                const unsigned int done = atomic_add_acq_rel(f.row_cnt + g.r, 1u) + 1u;
+                sm.last_of[tid] = done == (unsigned int)(cl - cf + 1);
+            }
+        }
         __syncthreads();
-        if (tid == 0) f.num_selected[r] = kb;
-        select_row<kThreads>(keys, NB, p.kmax, f.block_idx + (size_t)r * p.kmax, sm.sel);
+        // the rows this CTA completes: load their keys, then the CTA selects each
+        SelectSmem<kThreads>& ssm = *reinterpret_cast<SelectSmem<kThreads>*>(m.base + f.chunk_off);
+        for (int k = 0; k < nb; ++k) {
+            if (!sm.last_of[k]) continue;
+            const GateRow& g = sm.rows[k];
+            if (g.scored && !whole_rows)
+                for (int i = tid; i < g.NB - 1; i += kThreads) keys[i] = __ldcg(f.keys_g + (size_t)g.r * f.NBmax + i);
+            if (tid == 0) {
+                f.num_selected[g.r] = p.kmax < g.NB ? p.kmax : g.NB;
+                f.row_cnt[g.r] = 0u;   // ready for the next call: every reader of the row's
+                f.qg_flag[g.r] = 0u;   // projected query has counted in by now
+            }
+            __syncthreads();
+            select_row<kThreads>(keys, g.NB, p.kmax, f.block_idx + (size_t)g.r * p.kmax, ssm);
+            __syncthreads();
+        }
         fence_proxy_async_smem();
-        __syncthreads();  // scratch and keys are reused by the next row
+        __syncthreads();  // scratch, keys and stages are reused by the next batch
+        r += nb;
     }
 }
 
@@ -670,25 +902,26 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& m) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
+        unsigned int* genp = bar + 32;  // the generation word sits on its own 128-byte line
         unsigned int gen;
-        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(gen) : "l"(genp) : "memory");
         const unsigned int arrived = atomicAdd(bar, 1u);
         bool ok = true;
         if (arrived == gridDim.x - 1) {
             atomicExch(bar, 0u);
             __threadfence();
-            atomicAdd(bar + 1, 1u);
+            atomicAdd(genp, 1u);
         } else {
             const uint64_t t0 = global_timer_ns();
             while (true) {
                 unsigned int now;
-                asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(now) : "l"(bar + 1) : "memory");
+                asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(now) : "l"(genp) : "memory");
                 if (now != gen) break;
                 if (global_timer_ns() - t0 > kWaitLimitNs) {
                     ok = false;
                     break;
                 }
-                __nanosleep(64);
+                __nanosleep(256);  // ~140 waiters: keep the line's L2 slice free for real traffic
             }
         }
         __threadfence();
@@ -699,7 +932,7 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& m) {
 }
 
 template <int D, int BLK, int DG>
-__global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registers as 12: <= 168 each
+__global__ void __launch_bounds__(kStepThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const Params p, const StepParams f) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -714,7 +947,9 @@ __global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registe
     if ((int)blockIdx.x >= p.P) return;  // more SMs than decode ranges
     const long long g0 = (long long)blockIdx.x * p.V / p.P;
     const long long g1 = (long long)(blockIdx.x + 1) * p.V / p.P;
-    if ((threadIdx.x >> 5) == kConsumerWarps) decode_producer<D, BLK, true>(&tmK, &tmV, p, m, g0, g1);
+    const int warp = threadIdx.x >> 5;
+    if (warp == kConsumerWarps) decode_producer<D, BLK, true>(&tmK, &tmV, p, m, g0, g1);
+    else if (warp >= kHelperWarp0) decode_helpers<D, BLK>(p, f, m, g0, g1);
     else decode_consumers<D, BLK, true>(p, f, m, g0, g1);
 }
 
@@ -737,23 +972,25 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns) {
 // ---------------------------------------------------------------- host side
 
 struct Layout {
-    int nst, stage_bytes, merge_off, info_off, bar_off, total;
+    int nst, stage_bytes, merge_off, info_off, bar_off, refresh_off, total;
 };
 
 template <int D, int BLK>
-Layout make_layout(int G) {
+Layout make_layout(int G, bool with_refresh) {
     using C = Cfg<D, BLK>;
     Layout l;
     l.stage_bytes = (2 * C::kTileBytes + G * D * 2 + 1023) / 1024 * 1024;
     const int merge_bytes = kConsumerWarps * G * D * 4 + 2 * kConsumerWarps * G * 4;
-    const int bar_bytes = (2 * kMaxStages + 1 + kMaxGateStages) * 8;
-    const int tail = merge_bytes + kInfoWords * 4 + bar_bytes + 64;
+    const int bar_bytes = (2 * kMaxStages + 2 + kMaxGateStages) * 8;
+    const int refresh_bytes = with_refresh ? (int)sizeof(PoolSmem<D>) + 16 : 0;
+    const int tail = merge_bytes + kInfoWords * 4 + bar_bytes + refresh_bytes + 64;
     int nst = (kSmemLimit - 1024 - tail) / l.stage_bytes;
     l.nst = nst > kMaxStages ? kMaxStages : nst;
     l.merge_off = l.nst * l.stage_bytes;
     l.info_off = (l.merge_off + merge_bytes + 15) / 16 * 16;
     l.bar_off = (l.info_off + kInfoWords * 4 + 15) / 16 * 16;
-    l.total = l.bar_off + bar_bytes + 1024;  // + slack for the 1024-byte alignment
+    l.refresh_off = l.bar_off + bar_bytes;
+    l.total = l.refresh_off + refresh_bytes + 1024;  // + slack for the 1024-byte alignment
     return l;
 }
 
@@ -791,7 +1028,7 @@ cudaError_t allow_big_smem(K kernel) {
 template <int D, int BLK>
 cudaError_t launch_impl(const Shape& s, const DecodeLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
                         int num_sms, cudaStream_t stream) {
-    const Layout l = make_layout<D, BLK>(s.G);
+    const Layout l = make_layout<D, BLK>(s.G, false);
     if (l.nst < 2) return cudaErrorInvalidConfiguration;
     static bool attr_done = false;  // once per template instance (benign race)
     if (!attr_done) {
@@ -813,7 +1050,7 @@ int step_num_splits(const Shape& s, int kmax, int num_sms) {
 template <int D, int BLK, int DG>
 cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tmK, const CUtensorMap& tmV,
                       int num_sms, cudaStream_t stream) {
-    const Layout l = make_layout<D, BLK>(s.G);
+    const Layout l = make_layout<D, BLK>(s.G, true);
     if (l.nst < 2) return cudaErrorInvalidConfiguration;
     const int keys_bytes = (s.NBmax * 4 + 1023) / 1024 * 1024;
     const int ring = l.nst * l.stage_bytes;
@@ -856,15 +1093,21 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     f.lse_out = a.lse_out;
     f.grid_bar = reinterpret_cast<unsigned int*>(ws + wl.grid_bar);
     f.row_done = reinterpret_cast<unsigned int*>(ws + wl.row_done);
+    f.row_cnt = reinterpret_cast<unsigned int*>(ws + wl.row_cnt);
+    f.qg_flag = reinterpret_cast<unsigned int*>(ws + wl.qg_flag);
+    f.qg_g = reinterpret_cast<float*>(ws + wl.qg);
+    f.keys_g = reinterpret_cast<uint32_t*>(ws + wl.keys);
     f.rows = s.B * s.Hkv;
     f.NBmax = s.NBmax;
+    f.dg = s.dg;
+    f.refresh_off = l.refresh_off;
     f.keys_off = kGateScratchBytes;
     f.chunk_off = kGateScratchBytes + keys_bytes;
     f.n_gate_stages = n_gate > kMaxGateStages ? kMaxGateStages : n_gate;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms, 1, 1);  // every SM: phase 1 spreads rows over all of them
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kStepThreads, 1, 1);
     cfg.dynamicSmemBytes = l.total;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -886,7 +1129,12 @@ WorkspaceLayout step_workspace_layout(const Shape& s, int kmax, int num_sms) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     w.grid_bar = 0;
     w.row_done = 256;
-    w.o_part = up(w.row_done + rows * 4);
+    w.row_cnt = up(w.row_done + rows * 4);
+    w.qg_flag = up(w.row_cnt + rows * 4);
+    w.counters_end = up(w.qg_flag + rows * 4);  // everything before this must start at zero
+    w.qg = w.counters_end;
+    w.keys = up(w.qg + rows * (size_t)s.dg * 4);
+    w.o_part = up(w.keys + rows * (size_t)s.NBmax * 4);
     w.lse_part = up(w.o_part + (size_t)s.B * s.Hq * S * s.D * 4);
     w.total = up(w.lse_part + (size_t)s.B * s.Hq * S * 4);
     return w;
@@ -960,7 +1208,7 @@ cudaError_t launch_decode_step_static(const Shape& s, StepLaunch a, const CUtens
     if (wl.total > kStaticScratchBytes) return cudaErrorInvalidValue;
     // The array keeps the previous call's contents: the barrier words and row
     // counts must start at zero.
-    e = cudaMemsetAsync(scratch[dev], 0, wl.o_part, stream);
+    e = cudaMemsetAsync(scratch[dev], 0, wl.counters_end, stream);
     if (e != cudaSuccess) return e;
     a.workspace = scratch[dev];
     return launch_decode_step(s, a, tmK, tmV, num_sms, stream);
