@@ -41,7 +41,9 @@ DEFAULT_WORKLOAD = "decode_b16"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sparse_decode_traffic.json")
-DECODE_SRC = os.path.join(ROOT, "block_sparse_attention_seer_b200", "csrc", "sparse_decode.cu")
+# the sources the fused step kernel is compiled from: a recorded traffic figure holds only while they are unchanged
+DECODE_SRCS = [os.path.join(ROOT, "block_sparse_attention_seer_b200", "csrc", f)
+               for f in ("sparse_decode.cu", "gate_core.cuh", "seer_device.cuh")]
 
 
 def parse():
@@ -97,13 +99,20 @@ def algorithmic_bytes(wl, seq_lens, block_idx, num_selected):
     return kv + kp + qo, kv + qo // 2, toks, blocks
 
 
+def kernel_sources_sha256():
+    h = hashlib.sha256()
+    for path in DECODE_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def recorded_traffic(kernel_launch_bytes_scale=1.0):
     """DRAM traffic per decode launch from the committed ncu summary, if the kernel is unchanged."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
-        src = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
-        if d.get("source_sha256") != src:
+        if d.get("sources_sha256") != kernel_sources_sha256():
             return None
         return d
     except Exception:

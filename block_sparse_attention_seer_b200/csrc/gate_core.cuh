@@ -170,73 +170,95 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 // ---------------------------------------------------------------- selection
+//
+// The block list of a row is its last block NB-1 plus the m = kb - 1 largest
+// keys among candidates 0 .. NB-2, in the order "larger key first, equal keys
+// by lower index". That set is fixed by its last member T = (kT, iT):
+// candidate i is kept iff key_i > kT, or key_i == kT and i <= iT.
 
-// ---------------------------------------------------------------- selection
+constexpr int kSelectBins = 2048;
+constexpr int kSelectBucket = 64;  // boundary bins up to this size are ranked exactly
 
 template <int kThreads>
 struct SelectSmem {
-    int hist[4096];
-    int warp_tot[kThreads / 32];
-    int bucket, rem, nbound;
-    uint32_t bkey[32];  // keys of a boundary bucket of at most 32 elements
-    int bidx[32];
-    int taken[32];      // which of them are kept
+    alignas(16) int hist[kSelectBins];
+    alignas(16) uint32_t bkey[kSelectBucket];
+    alignas(16) int bidx[kSelectBucket];
+    uint32_t wlo[kThreads / 32], whi[kThreads / 32];
+    int wsum[kThreads / 32];
+    int bstar, bcount, above, bfill;
+    uint32_t kT;
+    int iT;
 };
 
-// Exclusive CTA-wide prefix sum of one value per thread (ascending thread
-// order); *total gets the sum.
-template <int kThreads>
-__device__ __forceinline__ int block_exclusive_scan(int v, SelectSmem<kThreads>& sm, int& total) {
-    constexpr int kWarps = kThreads / 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+__device__ __forceinline__ int warp_inclusive_scan(int x) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) sm.warp_tot[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int t = lane < kWarps ? sm.warp_tot[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += y;
-        }
-        if (lane < kWarps) sm.warp_tot[lane] = t;  // inclusive warp totals
-    }
-    __syncthreads();
-    total = sm.warp_tot[kWarps - 1];
-    const int before = warp == 0 ? 0 : sm.warp_tot[warp - 1];
-    __syncthreads();  // warp_tot is reused by the next scan
-    return before + x - v;
+    return x;
 }
+
+// Float value of an order key (inverse of order_key; key 0 gives NaN).
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Histogram bins over a key range [lo, hi], lo < hi: linear in the float value
+// when both ends, their difference and the scale are finite, else linear in
+// the key. Either way the bin is monotone in the key (k1 <= k2 => bin(k1) <=
+// bin(k2)), bin(lo) = 0 and bin(hi) > 0, so the keys of one bin form a key
+// interval that holds fewer distinct keys than [lo, hi].
+struct SelectBins {
+    uint32_t lo;
+    float flo, scale;
+    int shift;
+    bool by_value;
+    __device__ __forceinline__ void set(uint32_t lo_, uint32_t hi_) {
+        lo = lo_;
+        flo = key_value(lo_);
+        const float fhi = key_value(hi_);
+        const float w = fhi - flo;
+        scale = (float)kSelectBins / w;
+        by_value = isfinite(flo) && isfinite(fhi) && isfinite(w) && w > 0.f && isfinite(scale);
+        const uint32_t d = hi_ - lo_;
+        shift = max(0, 32 - __clz((int)d) - 11);  // (d >> shift) < kSelectBins
+    }
+    __device__ __forceinline__ int operator()(uint32_t k) const {
+        if (by_value) return min(kSelectBins - 1, (int)((key_value(k) - flo) * scale));
+        return (int)((k - lo) >> shift);
+    }
+};
 
 // Block list of one row. keys[0 .. NB-2] (shared memory) hold the order keys
 // of the candidate blocks 0 .. NB-2. Writes the kept indices in ascending
 // order to out[0 .. kb-1] (kb = min(kmax, NB): block NB-1 always, plus the
 // kb-1 largest keys, equal keys going to the lower index) and -1 to out[kb ..
-// kmax). Every thread of the CTA must call it.
+// kmax). Every thread of the CTA calls it; shared memory is reused only after
+// a barrier that follows the call.
 //
-// Radix select from the top with digits of 12, 12 and 8 bits: a histogram of
-// the current digit over the keys that match the prefix so far, a CTA scan
-// from the largest bucket down to the bucket holding the m-th largest key.
-// Block scores spread over many 12-bit buckets, so usually after the first
-// pass the boundary bucket holds at most 32 keys: one warp then sorts them
-// exactly (key descending, index ascending) and the rest is a compaction in
-// index order. Keys that stay equal over all 32 bits are resolved by index.
+// T is found by narrowing a key range [lo, hi] known to hold it: a histogram
+// of the range (SelectBins), a CTA scan of the bins from the top to the bin
+// where the count reaches the number still to take, then an exact ranking of
+// that bin when it holds at most kSelectBucket keys, else a new range = its
+// smallest and largest key. Every step removes at least one distinct key; a
+// range of one key value keeps its lowest indices. The common case is a
+// single histogram and seven barriers.
 template <int kThreads>
 __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __restrict__ out,
                            SelectSmem<kThreads>& sm) {
     constexpr int kWarps = kThreads / 32;
+    constexpr unsigned kFull = 0xffffffffu;
+    constexpr int kBinsPer = (kSelectBins + kThreads - 1) / kThreads;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kb = kmax < NB ? kmax : NB;
     for (int p = (kb > 0 ? kb : 0) + tid; p < kmax; p += kThreads) out[p] = -1;
     if (NB == 0) return;
-    const int ncand = NB - 1;  // blocks 0 .. NB-2 compete; NB-1 is always kept
-    const int m = kb - 1;      // how many of them to keep
-    if (m >= ncand) {          // everything fits in the budget
+    const int ncand = NB - 1;
+    const int m = kb - 1;
+    if (m >= ncand) {
         for (int j = tid; j < NB; j += kThreads) out[j] = j;
         return;
     }
@@ -244,125 +266,156 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
         if (tid == 0) out[0] = NB - 1;
         return;
     }
-    uint32_t prefix = 0, mask = 0;
-    int rem = m;          // how many keys still to take inside the current prefix
-    bool exact = false;   // boundary resolved by the warp sort
-    const int shifts[3] = {20, 8, 0};
-    const int widths[3] = {12, 12, 8};
-    for (int pass = 0; pass < 3 && !exact; ++pass) {
-        const int shift = shifts[pass];
-        const int nbins = 1 << widths[pass];
-        const uint32_t dmask = (uint32_t)nbins - 1u;
-        for (int i = tid; i < nbins; i += kThreads) sm.hist[i] = 0;
+    // Thread t owns the bins kSelectBins-1 - (t*kBinsPer + q), q < kBinsPer (from the top),
+    // the strided candidates t, t + kThreads, ... for order-free passes, and the
+    // contiguous candidates [c0, c1) for the passes in index order.
+    const int per = (ncand + kThreads - 1) / kThreads;
+    const int c0 = min(ncand, tid * per), c1 = min(ncand, c0 + per);
+    auto bin_of_q = [&](int q) { return kSelectBins - 1 - (tid * kBinsPer + q); };
+    auto clear_bins = [&]() {
+#pragma unroll
+        for (int q = 0; q < kBinsPer; ++q)
+            if (bin_of_q(q) >= 0) sm.hist[bin_of_q(q)] = 0;
+    };
+    // CTA min / max (one barrier; wlo / whi are read again only after later barriers)
+    auto block_min_max = [&](uint32_t a, uint32_t b, uint32_t& glo, uint32_t& ghi) {
+        a = __reduce_min_sync(kFull, a);
+        b = __reduce_max_sync(kFull, b);
+        if (lane == 0) {
+            sm.wlo[warp] = a;
+            sm.whi[warp] = b;
+        }
         __syncthreads();
+        glo = __reduce_min_sync(kFull, lane < kWarps ? sm.wlo[lane] : 0xffffffffu);
+        ghi = __reduce_max_sync(kFull, lane < kWarps ? sm.whi[lane] : 0u);
+    };
+    // exclusive CTA prefix sum in thread order (one barrier); the total to every thread
+    auto block_scan = [&](int v, int& total) {
+        const int x = warp_inclusive_scan(v);
+        if (lane == 31) sm.wsum[warp] = x;
+        __syncthreads();
+        const unsigned w = lane < kWarps ? (unsigned)sm.wsum[lane] : 0u;
+        total = (int)__reduce_add_sync(kFull, w);
+        return (int)__reduce_add_sync(kFull, lane < warp ? w : 0u) + x - v;
+    };
+
+    clear_bins();
+    if (tid == 0) sm.bfill = 0;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = tid; i < ncand; i += kThreads) {
+        lo = min(lo, keys[i]);
+        hi = max(hi, keys[i]);
+    }
+    block_min_max(lo, hi, lo, hi);
+    int rem = m;  // how many of the keys inside [lo, hi] are kept
+    uint32_t kT;
+    int iT;
+    while (true) {
+        if (lo == hi) {  // one key value left: its rem lowest indices
+            int c = 0;
+            for (int i = c0; i < c1; ++i) c += keys[i] == lo;
+            int total;
+            const int ex = block_scan(c, total);
+            if (ex < rem && rem <= ex + c) {
+                int seen = ex;
+                for (int i = c0; i < c1; ++i)
+                    if (keys[i] == lo && ++seen == rem) sm.iT = i;
+            }
+            __syncthreads();
+            kT = lo;
+            iT = sm.iT;
+            break;
+        }
+        SelectBins bins;
+        bins.set(lo, hi);
         for (int i = tid; i < ncand; i += kThreads) {
             const uint32_t k = keys[i];
-            if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & dmask], 1);
+            if (k >= lo && k <= hi) atomicAdd(&sm.hist[bins(k)], 1);
         }
         __syncthreads();
-        // thread t owns a run of bins counted from the top: bins nbins-1-t*per ... downwards
-        const int per = (nbins + kThreads - 1) / kThreads;
         int mine = 0;
-        for (int q = 0; q < per; ++q) {
-            const int bin = nbins - 1 - (tid * per + q);
-            if (bin >= 0) mine += sm.hist[bin];
-        }
+#pragma unroll
+        for (int q = 0; q < kBinsPer; ++q)
+            if (bin_of_q(q) >= 0) mine += sm.hist[bin_of_q(q)];
         int total;
-        const int above = block_exclusive_scan<kThreads>(mine, sm, total);
-        if (above < rem && rem <= above + mine) {
-            int run = above;
-            for (int q = 0; q < per; ++q) {
-                const int bin = nbins - 1 - (tid * per + q);
-                const int c = sm.hist[bin];
+        const int ex = block_scan(mine, total);
+        if (ex < rem && rem <= ex + mine) {
+            int run = ex;
+            for (int q = 0; q < kBinsPer && bin_of_q(q) >= 0; ++q) {
+                const int c = sm.hist[bin_of_q(q)];
                 if (run + c >= rem) {
-                    sm.bucket = bin;
-                    sm.rem = rem - run;
-                    sm.nbound = c;
+                    sm.bstar = bin_of_q(q);
+                    sm.bcount = c;
+                    sm.above = run;
                     break;
                 }
                 run += c;
             }
         }
         __syncthreads();
-        prefix |= (uint32_t)sm.bucket << shift;
-        mask |= dmask << shift;
-        rem = sm.rem;
-        const int nbound = sm.nbound;
-        __syncthreads();
-        if (nbound <= 32 && pass < 2) {
-            // gather the boundary bucket and sort it exactly inside one warp
-            if (tid == 0) sm.nbound = 0;
-            __syncthreads();
+        const int bstar = sm.bstar, bcount = sm.bcount;
+        rem -= sm.above;
+        if (bcount <= kSelectBucket) {
+            // gather the bin, then rank each entry against the others: T has rank rem - 1
             for (int i = tid; i < ncand; i += kThreads) {
                 const uint32_t k = keys[i];
-                if ((k & mask) == prefix) {
-                    const int at = atomicAdd(&sm.nbound, 1);
+                if (k >= lo && k <= hi && bins(k) == bstar) {
+                    const int at = atomicAdd(&sm.bfill, 1);
                     sm.bkey[at] = k;
                     sm.bidx[at] = i;
                 }
             }
             __syncthreads();
-            if (warp == 0) {
-                uint32_t k = lane < nbound ? sm.bkey[lane] : 0u;
-                int ix = lane < nbound ? sm.bidx[lane] : 0x7fffffff;
-                // bitonic sort of 32 (key, index): larger key first, then lower index; padding last
-#pragma unroll
-                for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-                    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                        const uint32_t ok = __shfl_xor_sync(0xffffffffu, k, stride);
-                        const int oi = __shfl_xor_sync(0xffffffffu, ix, stride);
-                        const bool mine_first = (k > ok) || (k == ok && ix < oi);
-                        const bool up = ((lane & size) == 0) == ((lane & stride) == 0);
-                        if (mine_first != up) {
-                            k = ok;
-                            ix = oi;
-                        }
-                    }
+            if (tid < bcount) {
+                const uint32_t mk = sm.bkey[tid];
+                const int mi = sm.bidx[tid];
+                int rank = 0;
+                for (int q = 0; q < bcount; ++q) {
+                    const uint32_t ok = sm.bkey[q];
+                    rank += ok > mk || (ok == mk && sm.bidx[q] < mi);
                 }
-                sm.taken[lane] = (lane < rem) ? ix : -1;  // the first `rem` of the sorted bucket
+                if (rank == rem - 1) {
+                    sm.kT = mk;
+                    sm.iT = mi;
+                }
             }
             __syncthreads();
-            exact = true;
+            kT = sm.kT;
+            iT = sm.iT;
+            break;
         }
+        // narrow to the bin's own key range; its bins are cleared for the next step
+        clear_bins();
+        uint32_t nlo = 0xffffffffu, nhi = 0u;
+        for (int i = tid; i < ncand; i += kThreads) {
+            const uint32_t k = keys[i];
+            if (k >= lo && k <= hi && bins(k) == bstar) {
+                nlo = min(nlo, k);
+                nhi = max(nhi, k);
+            }
+        }
+        block_min_max(nlo, nhi, lo, hi);
     }
-    // ---- compaction in index order (thread t owns a contiguous range of candidates)
-    const uint32_t tau = prefix;  // keys above the boundary prefix are kept
-    auto above_bound = [&](uint32_t k) { return (k & mask) > tau; };
-    auto kept = [&](int i, uint32_t k, int& eq_seen) {
-        if (above_bound(k)) return true;
-        if ((k & mask) != tau) return false;
-        if (exact) {
-#pragma unroll 4
-            for (int q = 0; q < 32; ++q)
-                if (sm.taken[q] == i) return true;
-            return false;
-        }
-        return eq_seen++ < rem;  // all 32 bits equal: the lowest indices win
+    // ---- compaction in index order
+    auto kept = [&](int i) {
+        const uint32_t k = keys[i];
+        return k > kT || (k == kT && i <= iT);
     };
-    const int per = (ncand + kThreads - 1) / kThreads;
-    const int i_lo = tid * per;
-    const int i_hi = min(ncand, i_lo + per);
-    int total;
-    int eq_before = 0;
-    if (!exact) {
-        int n_eq = 0;
-        for (int i = i_lo; i < i_hi; ++i) n_eq += (keys[i] & mask) == tau;
-        eq_before = block_exclusive_scan<kThreads>(n_eq, sm, total);
-    }
     int n_sel = 0;
     {
-        int eq = eq_before;
-        for (int i = i_lo; i < i_hi; ++i) n_sel += kept(i, keys[i], eq);
+        const int len = c1 - c0;  // read from a rotated start, so the lanes of a warp hit different banks
+        int off = len > 0 ? lane % len : 0;
+        for (int q = 0; q < len; ++q) {
+            n_sel += kept(c0 + off);
+            if (++off == len) off = 0;
+        }
     }
-    int pos = block_exclusive_scan<kThreads>(n_sel, sm, total);
-    {
-        int eq = eq_before;
-        for (int i = i_lo; i < i_hi; ++i)
-            if (kept(i, keys[i], eq)) out[pos++] = i;
-    }
+    int total;
+    int pos = block_scan(n_sel, total);
+    if (n_sel > 0)
+        for (int i = c0; i < c1; ++i)
+            if (kept(i)) out[pos++] = i;
     if (tid == 0) out[m] = NB - 1;
-    (void)kWarps;
 }
 
 }  // namespace seer

@@ -161,6 +161,17 @@ __device__ __forceinline__ float warp_max(float v) {
 // across the warp). Lane 0 of the warp returns the dot through `sink`.
 // One lane's piece of a W-row . v dot (4 or 2 columns); every matvec of the
 // library goes through these, so equal inputs give equal bits.
+// Read-only vector loads that stay where they are written (volatile asm keeps
+// them ahead of the barriers that follow), for loads issued early on purpose.
+__device__ __forceinline__ void load_early(float4& x, const float* p) {
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                 : "l"(p));
+}
+__device__ __forceinline__ void load_early(float2& x, const float* p) {
+    asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(x.x), "=f"(x.y) : "l"(p));
+}
+
 __device__ __forceinline__ float piece_dot(const float4& w, const float* v) {
     return w.x * v[0] + w.y * v[1] + w.z * v[2] + w.w * v[3];
 }

@@ -6,10 +6,10 @@
 // highest-scoring blocks among 0 .. NB_b - 2 (k_b = min(budget/blk, NB_b)),
 // equal scores going to the lower index, written in ascending order.
 //
-// One CTA per row (select_row, gate_core.cuh). Scores become
-// order-preserving 32-bit keys in shared memory; a radix select from the top
-// (12-bit histogram, then an exact warp sort of the boundary bucket) finds the
-// kept set, and a scan in index order writes it, ascending by construction.
+// One CTA per row (select_row, gate_core.cuh): the scores become
+// order-preserving 32-bit keys in shared memory, a value histogram narrows
+// down the last kept key, and a scan in index order writes the kept set,
+// ascending by construction.
 #include "gate_core.cuh"
 #include "seer_launch.h"
 
@@ -38,8 +38,9 @@ __global__ void __launch_bounds__(kThreads)
 
 cudaError_t launch_select_blocks(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax,
                                  int32_t* block_idx, int32_t* num_selected, cudaStream_t stream) {
+    const int rows = s.B * s.Hkv;
     const size_t smem = (size_t)s.NBmax * sizeof(uint32_t);
-    if (smem > 16 * 1024) {  // above what is left beside the static histogram
+    if (smem > 16 * 1024) {  // more than the default limit safely leaves beside the static scratch
         static bool attr_done = false;
         if (!attr_done) {
             cudaError_t e = cudaFuncSetAttribute(select_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -48,8 +49,8 @@ cudaError_t launch_select_blocks(const Shape& s, const float* scores, const int3
             attr_done = true;
         }
     }
-    select_blocks_kernel<<<s.B * s.Hkv, kThreads, smem, stream>>>(scores, seq_lens, s.Hkv, s.Lmax, s.blk, s.NBmax,
-                                                                  kmax, block_idx, num_selected);
+    select_blocks_kernel<<<rows, kThreads, smem, stream>>>(scores, seq_lens, s.Hkv, s.Lmax, s.blk, s.NBmax, kmax,
+                                                           block_idx, num_selected);
     return cudaGetLastError();
 }
 

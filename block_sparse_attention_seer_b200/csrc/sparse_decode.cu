@@ -113,6 +113,7 @@ struct StepParams {
     float* qg_g;             // [rows, dg] projected queries, written by each row's first CTA
     uint32_t* keys_g;        // [rows, NBmax] order keys of the block scores
     int rows, NBmax, dg;
+    int gate_ctas;                           // CTAs of phase 1 (a multiple of rows when rows fit the grid)
     int keys_off, chunk_off, n_gate_stages;  // phase-1 layout inside the stage ring
     int refresh_off;                         // phase-2 pool scratch (outside the ring)
 };
@@ -653,10 +654,11 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) 
     const int quad = lane >> 2, qlane = lane & 3;
     const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
     const long long V1 = (long long)f.rows * f.NBmax;
-    // With no more rows than CTAs every CTA takes one whole row (no hand-offs:
-    // its keys stay in shared memory and it selects right after scoring);
-    // otherwise the positions are spread over every CTA.
-    const int G1 = f.rows <= (int)gridDim.x ? f.rows : (int)gridDim.x;
+    // With no more rows than CTAs each row goes to the same whole number of
+    // CTAs (one CTA per row needs no hand-offs: its keys stay in shared memory
+    // and it selects right after scoring); with more rows the positions are
+    // spread evenly over every CTA.
+    const int G1 = f.gate_ctas;
     if ((int)blockIdx.x >= G1) return;
     const long long h0 = (long long)blockIdx.x * V1 / G1;
     const long long h1 = (long long)(blockIdx.x + 1) * V1 / G1;
@@ -694,7 +696,7 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) 
                 const int o = min(warp + u * kWarps, total_q - 1);
                 const int k = owned_row(o), e = o % DG;
                 const int kvh = (r + k) % p.Hkv;
-                w[u] = *reinterpret_cast<const WVec*>(f.w_q + ((size_t)kvh * DG + e) * D + lane * kVecD);
+                load_early(w[u], f.w_q + ((size_t)kvh * DG + e) * D + lane * kVecD);
             }
         }
         if (tid < nb) {
@@ -1098,6 +1100,7 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     f.qg_g = reinterpret_cast<float*>(ws + wl.qg);
     f.keys_g = reinterpret_cast<uint32_t*>(ws + wl.keys);
     f.rows = s.B * s.Hkv;
+    f.gate_ctas = f.rows <= num_sms ? f.rows * (num_sms / f.rows) : num_sms;
     f.NBmax = s.NBmax;
     f.dg = s.dg;
     f.refresh_off = l.refresh_off;

@@ -2,7 +2,9 @@
 oracle's selection on the same fp32 scores (widened exactly to fp64) bit for
 bit -- including all-equal scores (lowest indices win), clusters that share
 high-order bits (more radix passes), duplicated values at the boundary and
-signed zeros."""
+signed zeros. Rows of up to 1024 candidates go through the single-warp
+select (16 candidates per lane up to 512, 32 above), longer ones through the
+CTA-wide radix select: the sizes straddle both switches."""
 import numpy as np
 import pytest
 import torch
@@ -35,12 +37,18 @@ CASES = {
     "few_values": lambda rng, n: rng.choice(np.array([0.1, 0.2, 0.3, -0.2], np.float32), n),
     "signed_zeros": lambda rng, n: rng.choice(np.array([0.0, -0.0, 1e-30, -1e-30], np.float32), n),
     "wide": lambda rng, n: (rng.standard_normal(n) * 10.0 ** rng.integers(-20, 20, n)).astype(np.float32),
+    # powers of two over many octaves: the key range narrows over several histogram steps
+    "geometric": lambda rng, n: (rng.choice([-1.0, 1.0], n) * 2.0 ** -rng.integers(0, 120, n)).astype(np.float32),
+    # a dense run of adjacent floats next to a few far outliers
+    "adjacent_ulps": lambda rng, n: np.where(rng.random(n) < 0.02, 1e30,
+                                             1.0 + rng.integers(0, 3 * n, n) * 2.0 ** -23).astype(np.float32),
 }
 
 
 @pytest.mark.parametrize("case", sorted(CASES))
-@pytest.mark.parametrize("nb,blk,budget_blocks", [(2, 64, 1), (33, 64, 8), (512, 64, 64), (1024, 128, 103),
-                                                  (4097, 64, 512)])
+@pytest.mark.parametrize("nb,blk,budget_blocks", [(2, 64, 1), (33, 64, 8), (512, 64, 64), (513, 64, 100),
+                                                  (514, 64, 100), (1024, 128, 103), (1025, 64, 300),
+                                                  (1026, 64, 700), (4097, 64, 512)])
 def test_select_matches_oracle(case, nb, blk, budget_blocks):
     rng = np.random.default_rng(nb * 7 + len(case))
     B, Hkv = 2, 3
