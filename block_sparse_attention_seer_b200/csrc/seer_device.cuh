@@ -171,6 +171,11 @@ __device__ __forceinline__ void load_early(float4& x, const float* p) {
 __device__ __forceinline__ void load_early(float2& x, const float* p) {
     asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(x.x), "=f"(x.y) : "l"(p));
 }
+__device__ __forceinline__ int load_early(const int32_t* p) {
+    int x;
+    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(x) : "l"(p));
+    return x;
+}
 
 __device__ __forceinline__ float piece_dot(const float4& w, const float* v) {
     return w.x * v[0] + w.y * v[1] + w.z * v[2] + w.w * v[3];

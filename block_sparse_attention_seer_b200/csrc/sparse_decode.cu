@@ -106,7 +106,7 @@ struct StepParams {
     int32_t* num_selected;  // idem
     __nv_bfloat16* out;
     float* lse_out;
-    unsigned int* grid_bar;  // {arrivals, generation}
+    unsigned int* grid_bar;  // 64-bit arrival counter (grows by gridDim.x per launch)
     unsigned int* row_done;  // [rows] finished decode slots per row
     unsigned int* row_cnt;   // [rows] finished phase-1 pieces per row
     unsigned int* qg_flag;   // [rows] the row's projected query is in qg_g
@@ -689,6 +689,13 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) 
             }
         const int total_q = own_rows * DG;  // outputs ordered by owned row, then e
         auto owned_row = [&](int o) { return own_first + o / DG; };
+        // lengths and update starts of the batch rows: independent loads, issued first
+        int len_raw = 0, upd_raw = -1;
+        if (tid < nb) {
+            const int b = (r + tid) / p.Hkv;
+            len_raw = load_early(p.seq_lens + b);
+            if (f.upd_start) upd_raw = load_early(f.upd_start + b);
+        }
         WVec w[kQBatch];
         if (total_q > 0) {
 #pragma unroll
@@ -704,9 +711,10 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) 
             g.r = r + tid;
             g.b = g.r / p.Hkv;
             g.kvh = g.r - g.b * p.Hkv;
-            g.L = clamp_len(p.seq_lens[g.b], p.Lmax);
+            g.L = clamp_len(len_raw, p.Lmax);
             g.NB = (g.L + BLK - 1) / BLK;
-            g.js = g.NB > 0 ? refresh_start_block(f, g.b, g.L, g.NB, BLK) : g.NB;
+            const int st0 = max(f.upd_start ? upd_raw : g.L - 1, 0);  // as refresh_start_block
+            g.js = g.NB > 0 ? min(st0 / BLK, g.NB) : g.NB;
         }
         for (int idx = tid; idx < nb * D; idx += kThreads) {
             const int k = idx / D, d = idx - k * D;
@@ -898,35 +906,32 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) 
     }
 }
 
-// Bounded barrier over every CTA of a cooperative launch: {count, generation}
-// in global memory, left at count 0 for the next call. False if it gave up.
+// Bounded barrier over every CTA of a cooperative launch. One 64-bit arrival
+// counter that only grows (every launch adds gridDim.x, from zero), so there
+// is no reset step: a CTA's target is the next multiple of gridDim.x above
+// the count it finds when it arrives, and the critical path is one atomic of
+// the last CTA plus one poll of the others. False if it gave up.
 __device__ bool grid_barrier(unsigned int* bar, const Smem& m) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        unsigned int* genp = bar + 32;  // the generation word sits on its own 128-byte line
-        unsigned int gen;
-        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(gen) : "l"(genp) : "memory");
-        const unsigned int arrived = atomicAdd(bar, 1u);
+        unsigned long long* ctr = reinterpret_cast<unsigned long long*>(bar);
+        unsigned long long old;
+        asm volatile("atom.add.acq_rel.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr) : "memory");
+        const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
         bool ok = true;
-        if (arrived == gridDim.x - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            atomicAdd(genp, 1u);
-        } else {
+        if (old + 1 != target) {
             const uint64_t t0 = global_timer_ns();
             while (true) {
-                unsigned int now;
-                asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(now) : "l"(genp) : "memory");
-                if (now != gen) break;
+                unsigned long long now;
+                asm volatile("ld.acquire.gpu.u64 %0, [%1];" : "=l"(now) : "l"(ctr) : "memory");
+                if (now >= target) break;
                 if (global_timer_ns() - t0 > kWaitLimitNs) {
                     ok = false;
                     break;
                 }
-                __nanosleep(256);  // ~140 waiters: keep the line's L2 slice free for real traffic
+                __nanosleep(32);
             }
         }
-        __threadfence();
         if (!ok) record_failure(m.info);
     }
     __syncthreads();
