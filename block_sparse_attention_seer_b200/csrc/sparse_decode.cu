@@ -519,8 +519,14 @@ __device__ void decode_consumers(const Params& p, const StepParams& f, const Sme
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mM[w * p.G + h]);
                 float* lse_dst = p.lse_part + (head0 + h) * p.S + s.slot;
+                const bool direct = kFused && s.nslots == 1;  // the row's only piece: straight to the output
                 if (M == -INFINITY) {
-                    if (d == 0) *lse_dst = -INFINITY;
+                    if (direct) {
+                        f.out[(head0 + h) * D + d] = __float2bfloat16(0.f);
+                        if (d == 0 && f.lse_out) f.lse_out[head0 + h] = -INFINITY;
+                    } else if (d == 0) {
+                        *lse_dst = -INFINITY;
+                    }
                     continue;
                 }
                 float wsum = 0.f, acc = 0.f;
@@ -533,16 +539,25 @@ __device__ void decode_consumers(const Params& p, const StepParams& f, const Sme
                         acc += e * mO[(size_t)(w * p.G + h) * D + d];
                     }
                 }
+                if (direct) {
+                    f.out[(head0 + h) * D + d] = __float2bfloat16(acc / wsum);
+                    if (d == 0 && f.lse_out) f.lse_out[head0 + h] = (M + log2f(wsum)) * kLn2;
+                    continue;
+                }
                 p.o_part[((head0 + h) * p.S + s.slot) * D + d] = acc / wsum;
                 if (d == 0) *lse_dst = (M + log2f(wsum)) * kLn2;
             }
             // the merge area is reused by the next segment
             if (!(ok = consumer_sync(m, cph))) break;
+        } else if (kFused && s.nslots == 1) {  // a row without tokens, in one piece
+            for (int idx = ctid; idx < p.G * D; idx += kConsumerThreads)
+                f.out[head0 * D + idx] = __float2bfloat16(0.f);
+            if (ctid < p.G && f.lse_out) f.lse_out[head0 + ctid] = -INFINITY;
         } else if (ctid < p.G) {
             p.lse_part[(head0 + ctid) * p.S + s.slot] = -INFINITY;  // no kept block in this piece
         }
         if constexpr (kFused) {
-            merge_row_if_last<D>(p, f, m, s, cph);
+            if (s.nslots > 1) merge_row_if_last<D>(p, f, m, s, cph);  // else written above
             ok = m.info[kInfoAbort] == 0;
         } else if (s.last) {
             const int rest = p.S - s.nslots;
@@ -1048,9 +1063,23 @@ cudaError_t launch_impl(const Shape& s, const DecodeLaunch& a, const CUtensorMap
     return cudaGetLastError();
 }
 
+// Decode CTAs of the fused step. With no more rows than SMs every row gets
+// the same whole number c of CTAs, so each CTA range is one piece of one row
+// (no row hand-over in the middle of a stream; c = 1 writes the output
+// directly); otherwise one CTA per SM over the positions laid end to end.
+int step_decode_ctas(const Shape& s, int kmax, int num_sms) {
+    const long long rows = (long long)s.B * s.Hkv;
+    const long long V = rows * kmax;
+    if (rows <= num_sms) {
+        long long c = num_sms / rows;
+        if (c > kmax) c = kmax;
+        return (int)(rows * c);
+    }
+    return (int)(num_sms < V ? num_sms : V);
+}
+
 int step_num_splits(const Shape& s, int kmax, int num_sms) {
-    const long long V = (long long)s.B * s.Hkv * kmax;
-    long long P = num_sms < V ? num_sms : V;
+    const long long P = step_decode_ctas(s, kmax, num_sms);
     return (int)(kmax < P ? kmax : P);
 }
 
@@ -1071,7 +1100,7 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     }
     const int kmax = a.budget_tokens / s.blk;
     const long long V = (long long)s.B * s.Hkv * kmax;
-    const int P = (int)(num_sms < V ? num_sms : V);
+    const int P = step_decode_ctas(s, kmax, num_sms);
     const int S = step_num_splits(s, kmax, num_sms);
     unsigned char* ws = static_cast<unsigned char*>(a.workspace);
     WorkspaceLayout wl = step_workspace_layout(s, kmax, num_sms);
