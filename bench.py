@@ -58,6 +58,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=200)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    p.add_argument("--dense-steps", type=int, default=30, help="timed steps of the dense baseline (0: skip)")
     return p.parse_args()
 
 
@@ -107,11 +108,14 @@ def kernel_sources_sha256():
     return h.hexdigest()
 
 
-def recorded_traffic(kernel_launch_bytes_scale=1.0):
-    """DRAM traffic per decode launch from the committed ncu summary, if the kernel is unchanged."""
+def recorded_traffic(workload=None):
+    """DRAM traffic per fused-step launch from the committed ncu summary: only for the workload it
+    was recorded for (full batch) and only while the kernel's sources are unchanged."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
+        if workload is not None and d.get("workload") != workload:
+            return None
         if d.get("sources_sha256") != kernel_sources_sha256():
             return None
         return d
@@ -386,7 +390,7 @@ def run_ours(args):
     step_bytes, dec_bytes, toks, blocks = algorithmic_bytes(wl, lens, bidx, nsel)
     peak, peak_kind = measured_peak()
     achieved = step_bytes / (ms_step * 1e-3) / 1e9
-    traffic = recorded_traffic()
+    traffic = recorded_traffic(wl.name)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "kernel": "decode_step_kernel",
                 "traffic": (traffic["dram_bytes_per_launch"] if traffic else None),
@@ -398,6 +402,34 @@ def run_ours(args):
                 "sparse_decode_bytes": dec_bytes,
                 "sparse_decode_gbs": round(dec_achieved, 1),
                 "sparse_decode_frac": round(dec_achieved / peak, 4)}
+
+    # ---- dense baseline: the same decode kernels over every block of every row (a4 + a5)
+    dense = None
+    if args.dense_steps > 0:
+        nbm = wl.nb_max
+        idx_d, ns_d = W.identity_block_list(lens, wl.num_kv_heads, wl.block_size, nbm)
+        idx_d = torch.from_numpy(idx_d).to(dev)
+        ns_d = torch.from_numpy(ns_d).to(dev)
+        d_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.dense_steps)]
+        for k in range(args.dense_steps + 3):
+            prepare()
+            evs = d_ev[k - 3] if k >= 3 else None
+            if evs:
+                evs[0].record(stream)
+            st.attend(inp["q"], inp["k_cache"], inp["v_cache"], inp["seq_lens"], idx_d, ns_d, nbm)
+            if evs:
+                evs[1].record(stream)
+        torch.cuda.synchronize()
+        dense_us = float(np.mean([e[0].elapsed_time(e[1]) for e in d_ev])) * 1e3
+        if world > 1:
+            (dense_us,) = max_over_ranks([dense_us], dev)
+        _, dense_bytes, dense_toks, _ = algorithmic_bytes(wl, lens, idx_d.cpu().numpy(), ns_d.cpu().numpy())
+        dense = {"decode_us": round(dense_us, 3), "kernels": "sparse_decode + combine over every block",
+                 "tokens": dense_toks, "bytes": dense_bytes,
+                 "gbs": round(dense_bytes / (dense_us * 1e-6) / 1e9, 1),
+                 "frac": round(dense_bytes / (dense_us * 1e-6) / 1e9 / peak, 4),
+                 "speedup_of_sparse_step": round(dense_us / (ms_step * 1e3), 3),
+                 "speedup_of_sparse_decode": round(dense_us / (sep_step_ms * 1e3 - float(gate_ms.mean()) * 1e3), 3)}
 
     # ---- end to end through the public API: host inputs in, host output out, every step
     e2e = None
@@ -458,6 +490,7 @@ def run_ours(args):
             "step_frac_of_8tbs": round(step_bytes / (ms_step * 1e-3) / 8e12, 4),
             "step_us_p50": round(float(np.median(step_ms)) * 1e3, 3),
             "separate_calls": separate,
+            "dense_baseline": dense,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
