@@ -721,6 +721,7 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m) 
                 load_early(w[u], f.w_q + ((size_t)kvh * DG + e) * D + lane * kVecD);
             }
         }
+
         if (tid < nb) {
             GateRow& g = sm.rows[tid];
             g.r = r + tid;
@@ -965,7 +966,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     }
     gate_phase<D, BLK, DG>(p, f, m);
     fence_proxy_async_smem();  // phase-1 use of the ring precedes phase-2 copies into it
-    grid_barrier(f.grid_bar, m);
+    // One CTA per row in both phases: CTA r selects row r and then decodes it,
+    // nothing crosses CTAs, and a CTA barrier is all phase 2 needs.
+    if (f.gate_ctas == f.rows && p.P == f.rows) __syncthreads();
+    else grid_barrier(f.grid_bar, m);
     if ((int)blockIdx.x >= p.P) return;  // more SMs than decode ranges
     const long long g0 = (long long)blockIdx.x * p.V / p.P;
     const long long g1 = (long long)(blockIdx.x + 1) * p.V / p.P;
