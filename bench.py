@@ -431,17 +431,24 @@ def run_ours(args):
                  "speedup_of_sparse_step": round(dense_us / (ms_step * 1e3), 3),
                  "speedup_of_sparse_decode": round(dense_us / (sep_step_ms * 1e3 - float(gate_ms.mean()) * 1e3), 3)}
 
-    # ---- end to end through the public API: host inputs in, host output out, every step
+    # ---- end to end through the public API: host inputs in, host output out, every step.
+    # The step's inputs (q and the new token's K/V rows) travel as one packed pinned buffer;
+    # seer_append_kv places the token in the caches, the fused step runs, out comes back.
     e2e = None
     if args.e2e_steps > 0:
         B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
-        q_h = inp["q"].cpu().pin_memory()
-        kn_h = inp["k_cache"][:, :, int(lens[0]) - 1, :].contiguous().cpu().pin_memory()
-        vn_h = inp["v_cache"][:, :, int(lens[0]) - 1, :].contiguous().cpu().pin_memory()
+        nq, nkv = B * Hq * D, B * Hkv * D
+        last = torch.from_numpy(np.maximum(lens.astype(np.int64) - 1, 0)).to(dev)
+        rows_b = torch.arange(B, device=dev)
+        kn = inp["k_cache"][rows_b, :, last, :]  # the token already in the cache: the step is unchanged
+        vn = inp["v_cache"][rows_b, :, last, :]
+        packed_h = torch.cat([inp["q"].reshape(-1), kn.reshape(-1), vn.reshape(-1)]).cpu().pin_memory()
+        stage = torch.empty_like(packed_h, device=dev)
+        q_d = stage[:nq].view(B, Hq, D)
+        kn_d = stage[nq:nq + nkv].view(B, Hkv, D)
+        vn_d = stage[nq + nkv:].view(B, Hkv, D)
         out_h = torch.empty(B, Hq, D, dtype=torch.bfloat16).pin_memory()
-        uniform = bool((lens == lens[0]).all())
-        pos = int(lens[0]) - 1
-        h2d = q_h.numel() * 2 + (kn_h.numel() + vn_h.numel()) * 2
+        h2d = packed_h.numel() * 2
         d2h = out_h.numel() * 2
         e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
         for k in range(args.e2e_steps + 5):
@@ -450,11 +457,9 @@ def run_ours(args):
             evs = e_ev[k - 5] if k >= 5 else None
             if evs:
                 evs[0].record(stream)
-            inp["q"].copy_(q_h, non_blocking=True)
-            if uniform:
-                inp["k_cache"][:, :, pos, :].copy_(kn_h, non_blocking=True)
-                inp["v_cache"][:, :, pos, :].copy_(vn_h, non_blocking=True)
-            run_fused()
+            stage.copy_(packed_h, non_blocking=True)
+            api.seer_append_kv(st.dims, kn_d, vn_d, inp["seq_lens"], inp["k_cache"], inp["v_cache"])
+            st.fused_step(q_d, inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
             out_h.copy_(st.out, non_blocking=True)
             if evs:
                 evs[1].record(stream)
@@ -463,7 +468,8 @@ def run_ours(args):
         if world > 1:
             (e2e_us,) = max_over_ranks([e2e_us], dev)
         e2e = {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h)}
+               "d2h_bytes_per_step": int(d2h),
+               "path": "one packed H2D (q, new K, new V) -> seer_append_kv -> seer_decode_step -> D2H of out"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -47,6 +47,7 @@ def _load_library():
         "seer_select_blocks": [D, P, P, I32, P, P, P],
         "seer_sparse_decode": [D, P, P, P, P, P, P, I32, I32, F32, P, P, P],
         "seer_combine": [D, P, P, I32, P, P, P],
+        "seer_append_kv": [D, P, P, P, P, P, P],
         "seer_default_num_splits": [I32, P],
         "seer_decode_wait_failures": [P, I32],
         "seer_decode_step_workspace_size": [D, I32, P],
@@ -134,6 +135,12 @@ def seer_sparse_decode(dims, q, k_cache, v_cache, seq_lens, block_idx, num_selec
 def seer_combine(dims, o_part, lse_part, num_splits, out, lse_out, stream=None):
     _check("seer_combine", LIB.seer_combine(ctypes.byref(dims), _ptr(o_part), _ptr(lse_part), int(num_splits),
                                             _ptr(out), _ptr(lse_out), _stream(stream)))
+
+
+def seer_append_kv(dims, k_new, v_new, seq_lens, k_cache, v_cache, stream=None):
+    """The step's token: K/V rows [B, Hkv, D] -> position L_b - 1 of the caches."""
+    _check("seer_append_kv", LIB.seer_append_kv(ctypes.byref(dims), _ptr(k_new), _ptr(v_new), _ptr(seq_lens),
+                                                _ptr(k_cache), _ptr(v_cache), _stream(stream)))
 
 
 def seer_decode_step_workspace_size(dims, budget_tokens) -> int:

@@ -180,6 +180,17 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
     return from_cuda(seer::launch_combine(s, o_part, lse_part, num_splits, out, lse_out, stream));
 }
 
+seer_status seer_append_kv(const seer_dims* dims, const void* k_new, const void* v_new, const int32_t* seq_lens,
+                           void* k_cache, void* v_cache, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!k_new || !v_new || !seq_lens || !k_cache || !v_cache) return SEER_ERR_INVALID_ARG;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+        return SEER_ERR_INVALID_ARG;
+    return from_cuda(seer::launch_append_kv(s, k_new, v_new, seq_lens, k_cache, v_cache, stream));
+}
+
 seer_status seer_decode_step_workspace_size(const seer_dims* dims, int32_t budget_tokens, size_t* bytes) {
     Shape s;
     seer_status st = check_dims(dims, s);

@@ -11,6 +11,8 @@
  *   a3 seer_select_blocks  the kept blocks under a token budget
  *   a4 seer_sparse_decode  split-KV flash-decode over the kept blocks only
  *   a5 seer_combine        merge of the split partials into the output
+ * and, around them: seer_append_kv (the step's token into the caches) and
+ * seer_decode_step (a1..a5 as one launch).
  *
  * Sources: "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
  * (abstract) for the decode setting, the un-pooled query, the token budget and
@@ -184,6 +186,26 @@ seer_status seer_sparse_decode(const seer_dims* dims, const void* q, const void*
  */
 seer_status seer_combine(const seer_dims* dims, const float* o_part, const float* lse_part,
                          int32_t num_splits, void* out, float* lse_out, cudaStream_t stream);
+
+/* Appending the step's token. "SeerAttention-R" (abstract) decodes
+ * auto-regressively: each step appends one token whose K and V take part in
+ * that same step. seer_append_kv writes the token's rows at position
+ * L_b - 1 of every (b, kv head) row of both caches (L_b = clamped
+ * seq_lens[b], the length AFTER the append; rows with L_b = 0 are left
+ * alone), so a caller ships q and the new K/V per step and no strided cache
+ * slices. Call it before the step on the same stream. No counterpart on the
+ * pages beyond the decode setting itself.
+ *
+ *   k_new, v_new  bf16 [B, Hkv, D]        (16-byte aligned)
+ *   seq_lens      int32 [B]
+ *   k_cache       bf16 [B, Hkv, Lmax, D]  (written at [b, kvh, L_b - 1, :])
+ *   v_cache       bf16 [B, Hkv, Lmax, D]  (idem)
+ *
+ * Errors: SEER_ERR_INVALID_ARG for NULL or unaligned pointers and invalid
+ * dims; SEER_ERR_UNSUPPORTED for head_dim outside {64, 128}.
+ */
+seer_status seer_append_kv(const seer_dims* dims, const void* k_new, const void* v_new, const int32_t* seq_lens,
+                           void* k_cache, void* v_cache, cudaStream_t stream);
 
 /*
  * The whole decode step, a1..a5, in ONE cooperative launch (one CTA per SM).

@@ -84,6 +84,17 @@ def test_null_pointers_and_bad_scalars_rejected():
     assert L.seer_default_num_splits(0, ctypes.byref(ctypes.c_int32())) == api.SEER_ERR_INVALID_ARG
 
 
+def test_append_kv_validates_on_host():
+    d = _dims()
+    L = api.LIB
+    assert L.seer_append_kv(None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_append_kv(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_append_kv(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_append_kv(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE + 8, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    bad = _dims(head_dim=96)
+    assert L.seer_append_kv(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, None) == api.SEER_ERR_UNSUPPORTED
+
+
 def test_python_wrapper_raises_on_error():
     with pytest.raises(api.SeerError) as e:
         api.seer_combine(_dims(head_dim=96), FAKE, FAKE, 4, FAKE, None, stream=0)
