@@ -55,8 +55,9 @@ def _load():
         lib.oracle_attend.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, ctypes.c_int32,
                                       ctypes.c_double, P, P]
         lib.oracle_merge.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, P, P]
+        lib.oracle_block_mass.argtypes = [ctypes.POINTER(_Dims), P, P, P, ctypes.c_double, P, P]
         for f in ("oracle_pool_project", "oracle_gate_scores", "oracle_select", "oracle_attend",
-                  "oracle_merge"):
+                  "oracle_merge", "oracle_block_mass"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -160,6 +161,26 @@ def attend(q_bits, k_bits, v_bits, seq_lens, block_idx, num_selected, block_size
     _load().oracle_attend(ctypes.byref(dm), qp, kp_, vp, slp, ip, np_, int(kmax), float(sm_scale),
                           out.ctypes.data_as(ctypes.c_void_p), lse.ctypes.data_as(ctypes.c_void_p))
     return out, lse
+
+
+def block_mass(q_bits, k_bits, seq_lens, block_size, sm_scale=0.0):
+    """Block-level ground truth: each query head's dense softmax mass per KV block.
+
+    q_bits uint16 [B, Hq, D]; k_bits uint16 [B, Hkv, Lmax, D]; seq_lens int32 [B].
+    Returns (mass float64 [B, Hq, NBmax] (0 past NB_b), lse float64 [B, Hq]).
+    """
+    q_bits, qp = _c(q_bits, np.uint16)
+    k_bits, kp_ = _c(k_bits, np.uint16)
+    B, Hq, D = q_bits.shape
+    _, Hkv, Lmax, _ = k_bits.shape
+    sl, slp = _c(seq_lens, np.int32)
+    nbmax = (Lmax + block_size - 1) // block_size
+    mass = np.empty((B, Hq, nbmax), np.float64)
+    lse = np.empty((B, Hq), np.float64)
+    dm = _dims(B, Hq, Hkv, D, 0, block_size, Lmax)
+    _load().oracle_block_mass(ctypes.byref(dm), qp, kp_, slp, float(sm_scale), mass.ctypes.data_as(ctypes.c_void_p),
+                              lse.ctypes.data_as(ctypes.c_void_p))
+    return mass, lse
 
 
 def merge(o_parts, lse_parts):

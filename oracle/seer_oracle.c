@@ -298,3 +298,49 @@ void oracle_merge(int32_t n_parts, int32_t D, const double* o_parts, const doubl
     for (int d = 0; d < D; ++d) out[d] /= wsum;
     *lse = M + log(wsum);
 }
+
+/* Block-level ground truth, [V1] (the customised attention that extracts the
+ * block-level target the gate is distilled from) read for one decode query:
+ * the dense softmax attention of each query head over all valid tokens, and
+ * the share of its probability that falls in each block.
+ *   z_t       = scale * q_h . K[b,kvh,t]            t < L_b (L_b clamped to [0, Lmax])
+ *   p_t       = exp(z_t) / sum_{t'} exp(z_t')
+ *   mass[j]   = sum_{t in block j, t < L_b} p_t      j < NB_b;  0 for j >= NB_b
+ *   lse       = log sum_t exp(z_t)                   (-inf when L_b = 0)
+ * Shapes: mass [B, Hq, NBmax], lse [B, Hq]. sm_scale <= 0 means 1/sqrt(D). */
+void oracle_block_mass(const oracle_dims* dm, const uint16_t* q, const uint16_t* k_cache,
+                       const int32_t* seq_lens, double sm_scale, double* mass, double* lse) {
+    const int B = dm->batch, Hq = dm->num_q_heads, Hkv = dm->num_kv_heads;
+    const int D = dm->head_dim, blk = dm->block_size, Lmax = dm->max_seq_len;
+    const int G = Hq / Hkv;
+    const int NBmax = num_blocks(Lmax, blk);
+    const double scale = (sm_scale > 0.0) ? sm_scale : 1.0 / sqrt((double)D);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int row = 0; row < B * Hkv; ++row) {
+        const int b = row / Hkv, kvh = row % Hkv;
+        int L = seq_lens[b];
+        L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
+        double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        for (int h = 0; h < G; ++h) {
+            const int hq = kvh * G + h;
+            const uint16_t* qh = q + ((size_t)b * Hq + hq) * D;
+            double* mh = mass + ((size_t)b * Hq + hq) * NBmax;
+            for (int j = 0; j < NBmax; ++j) mh[j] = 0.0;
+            if (L == 0) { lse[(size_t)b * Hq + hq] = -INFINITY; continue; }
+            double m = -INFINITY;
+            for (int t = 0; t < L; ++t) {
+                const uint16_t* kt = k_cache + ((size_t)row * Lmax + t) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += bf16_to_double(qh[d]) * bf16_to_double(kt[d]);
+                z[t] = acc * scale;
+                if (z[t] > m) m = z[t];
+            }
+            double denom = 0.0;
+            for (int t = 0; t < L; ++t) denom += exp(z[t] - m);
+            for (int t = 0; t < L; ++t) mh[t / blk] += exp(z[t] - m) / denom;
+            const double lse_h = m + log(denom);
+            lse[(size_t)b * Hq + hq] = lse_h;
+        }
+        free(z);
+    }
+}

@@ -39,6 +39,12 @@ MUTANTS = {
     "attend_reads_past_length": [("const int t1 = (j * blk + blk < L) ? j * blk + blk : L;\n            for (int t",
                                   "const int t1 = j * blk + blk;\n            for (int t")],
     "merge_weight_sign": [("const double w = exp(lse_parts[s] - M);", "const double w = exp(M - lse_parts[s]);")],
+    "block_mass_scale_dropped": [("z[t] = acc * scale;", "z[t] = acc;")],
+    "block_mass_next_block": [("mh[t / blk] += exp(z[t] - m) / denom;",
+                               "mh[(t + 1) / blk < NBmax ? (t + 1) / blk : t / blk] += exp(z[t] - m) / denom;")],
+    "block_mass_ignores_length": [("L = L < 0 ? 0 : (L > Lmax ? Lmax : L);\n        double* z",
+                                   "L = Lmax;\n        double* z")],
+    "block_mass_lse_missing_max": [("const double lse_h = m + log(denom);", "const double lse_h = log(denom);")],
     "value_row_of_wrong_head": [("const uint16_t* vt = v_cache + ((size_t)row * Lmax + tok[i]) * D;",
                                  "const uint16_t* vt = v_cache + ((size_t)(row ^ 1) * Lmax + tok[i]) * D;")],
 }

@@ -339,3 +339,67 @@ def test_merge_all_empty(oracle):
 
 def test_thread_count_reported(oracle):
     assert oracle.num_threads() >= 1
+
+
+# ---------------------------------------------------------------- block-level ground truth
+
+def test_block_mass_equals_torch_softmax_per_block(oracle):
+    # The block mass is the dense softmax of each query head (torch float64)
+    # summed over each block's valid tokens; lse is its log-denominator.
+    for seed, blk in ((0, 64), (1, 128)):
+        wl, c = small_case(seed, blk=blk)
+        mass, lse = oracle.block_mass(c["q"], c["k"], c["lens"], blk)
+        q, K = torch.from_numpy(widen(c["q"])), torch.from_numpy(widen(c["k"]))
+        G, D = wl.group, wl.head_dim
+        for b in range(wl.batch):
+            L = int(c["lens"][b])
+            NB = -(-L // blk)
+            for h in range(wl.num_q_heads):
+                z = (K[b, h // G, :L] @ q[b, h]) / math.sqrt(D)
+                p = torch.softmax(z, 0)
+                ref = torch.zeros(wl.nb_max, dtype=torch.float64)
+                ref.index_add_(0, torch.arange(L) // blk, p)
+                np.testing.assert_allclose(mass[b, h], ref.numpy(), rtol=0, atol=1e-13)
+                assert abs(lse[b, h] - torch.logsumexp(z, 0).item()) < 1e-12
+                assert np.all(mass[b, h, NB:] == 0.0)
+
+
+def test_block_mass_zero_keys_is_token_share(oracle):
+    # K = 0: uniform softmax, so block j holds n_j / L of the mass (the
+    # partial last block its own token count) and lse = ln L.
+    wl, c = small_case(5, lens=(300, 65))
+    c["k"][:] = bits(np.zeros(1, np.float32))[0]
+    mass, lse = oracle.block_mass(c["q"], c["k"], c["lens"], wl.block_size)
+    for b, L in enumerate(int(x) for x in c["lens"]):
+        n = [min(64, L - j * 64) for j in range(-(-L // 64))] + [0] * (wl.nb_max - (-(-L // 64)))
+        for h in range(wl.num_q_heads):
+            np.testing.assert_allclose(mass[b, h], np.array(n) / L, rtol=0, atol=1e-13)
+            assert abs(lse[b, h] - math.log(L)) < 1e-12
+
+
+def test_block_mass_constant_logit_per_block_closed_form(oracle):
+    # K rows equal c_j * e_0 inside block j and q = e_0: every logit of block j
+    # is c_j / sqrt(D), so mass_j = n_j exp(c_j / sqrt(D)) / sum_i n_i exp(c_i / sqrt(D)).
+    wl, c = small_case(6, lens=(320, 200))
+    D = wl.head_dim
+    cj = np.array([2.0, -1.0, 0.5, 4.0, -3.0], np.float32)
+    K = np.zeros((wl.batch, wl.num_kv_heads, wl.max_seq_len, D), np.float32)
+    for j, v in enumerate(cj):
+        K[:, :, j * 64:(j + 1) * 64, 0] = v
+    Q = np.zeros((wl.batch, wl.num_q_heads, D), np.float32)
+    Q[:, :, 0] = 1.0
+    mass, lse = oracle.block_mass(bits(Q), bits(K), c["lens"], 64)
+    for b, L in enumerate(int(x) for x in c["lens"]):
+        NB = -(-L // 64)
+        n = np.array([min(64, L - j * 64) for j in range(NB)], np.float64)
+        w = n * np.exp(cj[:NB].astype(np.float64) / math.sqrt(D))
+        for h in range(wl.num_q_heads):
+            np.testing.assert_allclose(mass[b, h, :NB], w / w.sum(), rtol=1e-13, atol=0)
+            assert abs(lse[b, h] - math.log(w.sum())) < 1e-12
+
+
+def test_block_mass_single_block_and_empty(oracle):
+    wl, c = small_case(7, lens=(40, 0))
+    mass, lse = oracle.block_mass(c["q"], c["k"], c["lens"], wl.block_size)
+    assert np.all(np.abs(mass[0, :, 0] - 1.0) < 1e-13) and np.all(mass[0, :, 1:] == 0.0)
+    assert np.all(mass[1] == 0.0) and np.all(lse[1] == -np.inf)
