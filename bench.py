@@ -59,6 +59,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--dense-steps", type=int, default=30, help="timed steps of the dense baseline (0: skip)")
+    p.add_argument("--mass-steps", type=int, default=30, help="timed calls of the block-level ground truth (0: skip)")
     return p.parse_args()
 
 
@@ -431,6 +432,30 @@ def run_ours(args):
                  "speedup_of_sparse_step": round(dense_us / (ms_step * 1e3), 3),
                  "speedup_of_sparse_decode": round(dense_us / (sep_step_ms * 1e3 - float(gate_ms.mean()) * 1e3), 3)}
 
+    # ---- block-level ground truth (seer_block_mass): each head's dense softmax mass per block
+    block_mass = None
+    if args.mass_steps > 0:
+        mass_buf = torch.empty(wl.batch, wl.num_q_heads, wl.nb_max, dtype=torch.float32, device=dev)
+        mlse_buf = torch.empty(wl.batch, wl.num_q_heads, dtype=torch.float32, device=dev)
+        m_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.mass_steps)]
+        for k in range(args.mass_steps + 3):
+            prepare()
+            evs = m_ev[k - 3] if k >= 3 else None
+            if evs:
+                evs[0].record(stream)
+            api.seer_block_mass(st.dims, inp["q"], inp["k_cache"], inp["seq_lens"], mass_buf, mlse_buf)
+            if evs:
+                evs[1].record(stream)
+        torch.cuda.synchronize()
+        mass_us = float(np.mean([e[0].elapsed_time(e[1]) for e in m_ev])) * 1e3
+        if world > 1:
+            (mass_us,) = max_over_ranks([mass_us], dev)
+        k_bytes = int(sum(min(int(L), wl.max_seq_len) for L in lens)) * wl.num_kv_heads * wl.head_dim * 2
+        mass_bytes = k_bytes + wl.batch * wl.num_q_heads * (wl.head_dim * 2 + wl.nb_max * 4 + 4)
+        block_mass = {"us": round(mass_us, 3), "kernels": "block_lse + block_mass_finalize",
+                      "bytes": mass_bytes, "gbs": round(mass_bytes / (mass_us * 1e-6) / 1e9, 1),
+                      "frac": round(mass_bytes / (mass_us * 1e-6) / 1e9 / peak, 4)}
+
     # ---- end to end through the public API: host inputs in, host output out, every step.
     # The step's inputs (q and the new token's K/V rows) travel as one packed pinned buffer;
     # seer_append_kv places the token in the caches, the fused step runs, out comes back.
@@ -497,6 +522,7 @@ def run_ours(args):
             "step_us_p50": round(float(np.median(step_ms)) * 1e3, 3),
             "separate_calls": separate,
             "dense_baseline": dense,
+            "block_mass": block_mass,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,

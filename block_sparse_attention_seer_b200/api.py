@@ -48,6 +48,7 @@ def _load_library():
         "seer_sparse_decode": [D, P, P, P, P, P, P, I32, I32, F32, P, P, P],
         "seer_combine": [D, P, P, I32, P, P, P],
         "seer_append_kv": [D, P, P, P, P, P, P],
+        "seer_block_mass": [D, P, P, P, F32, P, P, P],
         "seer_default_num_splits": [I32, P],
         "seer_decode_wait_failures": [P, I32],
         "seer_decode_step_workspace_size": [D, I32, P],
@@ -135,6 +136,12 @@ def seer_sparse_decode(dims, q, k_cache, v_cache, seq_lens, block_idx, num_selec
 def seer_combine(dims, o_part, lse_part, num_splits, out, lse_out, stream=None):
     _check("seer_combine", LIB.seer_combine(ctypes.byref(dims), _ptr(o_part), _ptr(lse_part), int(num_splits),
                                             _ptr(out), _ptr(lse_out), _stream(stream)))
+
+
+def seer_block_mass(dims, q, k_cache, seq_lens, mass, lse_out=None, sm_scale=0.0, stream=None):
+    """Each query head's dense softmax mass per KV block -> mass [B, Hq, NBmax], lse [B, Hq]."""
+    _check("seer_block_mass", LIB.seer_block_mass(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(seq_lens),
+                                                  float(sm_scale), _ptr(mass), _ptr(lse_out), _stream(stream)))
 
 
 def seer_append_kv(dims, k_new, v_new, seq_lens, k_cache, v_cache, stream=None):

@@ -180,6 +180,18 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
     return from_cuda(seer::launch_combine(s, o_part, lse_part, num_splits, out, lse_out, stream));
 }
 
+seer_status seer_block_mass(const seer_dims* dims, const void* q, const void* k_cache, const int32_t* seq_lens,
+                            float sm_scale, float* mass, float* lse_out, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !k_cache || !seq_lens || !mass) return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(mass, 4)) return SEER_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
+    const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
+    return from_cuda(seer::launch_block_mass(s, q, k_cache, seq_lens, scale, mass, lse_out, stream));
+}
+
 seer_status seer_append_kv(const seer_dims* dims, const void* k_new, const void* v_new, const int32_t* seq_lens,
                            void* k_cache, void* v_cache, cudaStream_t stream) {
     Shape s;

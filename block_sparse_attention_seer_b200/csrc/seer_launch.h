@@ -80,6 +80,11 @@ cudaError_t launch_decode_step_static(const Shape& s, StepLaunch a, const CUtens
 cudaError_t read_decode_wait_failures(unsigned int* count, bool reset);
 cudaError_t run_wait_selftest(unsigned long long limit_ns, int* timed_out);
 
+// Block-level ground truth: each query head's dense softmax mass per KV block
+// [B, Hq, NBmax] and lse [B, Hq] (nullable) (block_mass.cu).
+cudaError_t launch_block_mass(const Shape& s, const void* q, const void* k_cache, const int32_t* seq_lens,
+                              float sm_scale, float* mass, float* lse_out, cudaStream_t stream);
+
 // New token's K and V rows [B, Hkv, D] -> position L_b - 1 of the caches (append_kv.cu).
 cudaError_t launch_append_kv(const Shape& s, const void* k_new, const void* v_new, const int32_t* seq_lens,
                              void* k_cache, void* v_cache, cudaStream_t stream);

@@ -11,8 +11,9 @@
  *   a3 seer_select_blocks  the kept blocks under a token budget
  *   a4 seer_sparse_decode  split-KV flash-decode over the kept blocks only
  *   a5 seer_combine        merge of the split partials into the output
- * and, around them: seer_append_kv (the step's token into the caches) and
- * seer_decode_step (a1..a5 as one launch).
+ * and, around them: seer_append_kv (the step's token into the caches),
+ * seer_decode_step (a1..a5 as one launch) and seer_block_mass (the gate's
+ * block-level ground truth).
  *
  * Sources: "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning"
  * (abstract) for the decode setting, the un-pooled query, the token budget and
@@ -186,6 +187,30 @@ seer_status seer_sparse_decode(const seer_dims* dims, const void* q, const void*
  */
 seer_status seer_combine(const seer_dims* dims, const float* o_part, const float* lse_part,
                          int32_t num_splits, void* out, float* lse_out, cudaStream_t stream);
+
+/* Block-level ground truth of one decode query. "SeerAttention: Learning
+ * Intrinsic Sparse Attention in Your LLMs" (abstract) distils its gate from a
+ * block-level ground truth extracted by a customised attention kernel; read
+ * for a decode query it is the share of each query head's dense softmax that
+ * falls in each KV block:
+ *   z_t = sm_scale * q_h . K[b, kvh, t],  t < L_b (L_b = clamped seq_lens[b])
+ *   mass[b, h, j] = sum_{t in block j} exp(z_t) / sum_t exp(z_t)   (j < NB_b)
+ *   mass[b, h, j] = 0                                               (j >= NB_b)
+ *   lse_out[b, h] = log sum_t exp(z_t)        (-inf when L_b = 0; mass all 0)
+ * sm_scale <= 0 means 1/sqrt(head_dim). Two launches (per-block log-masses
+ * into `mass`, then a per-row normalisation in place); reads all of K once.
+ *
+ *   q        bf16 [B, Hq, D]            (16-byte aligned)
+ *   k_cache  bf16 [B, Hkv, Lmax, D]     (16-byte aligned)
+ *   seq_lens int32 [B]
+ *   mass     fp32 [B, Hq, NBmax]        (output)
+ *   lse_out  fp32 [B, Hq]               (output, may be NULL)
+ *
+ * Errors: SEER_ERR_INVALID_ARG for NULL/unaligned pointers, a NaN or infinite
+ * sm_scale or invalid dims; SEER_ERR_UNSUPPORTED outside the supported sizes.
+ */
+seer_status seer_block_mass(const seer_dims* dims, const void* q, const void* k_cache, const int32_t* seq_lens,
+                            float sm_scale, float* mass, float* lse_out, cudaStream_t stream);
 
 /* Appending the step's token. "SeerAttention-R" (abstract) decodes
  * auto-regressively: each step appends one token whose K and V take part in
