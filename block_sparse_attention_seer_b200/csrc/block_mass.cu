@@ -11,9 +11,9 @@
 //   lse     = log sum_t exp(z_t)
 //
 // Pass 1 (block_lse_kernel): one warp per KV block. The warp copies the
-// block's K tile into its own shared-memory buffer with 16-byte cp.async
-// (rows padded by 16 bytes so that ldmatrix reads are conflict-free),
-// double-buffered across the warp's blocks, computes Q K^T on the tensor
+// block's K tile, 64 tokens at a time, into its own shared-memory ring with
+// 16-byte cp.async (rows padded by 16 bytes so that ldmatrix reads are
+// conflict-free; three stages, two tiles in flight), computes Q K^T on the tensor
 // cores (mma.sync bf16 -> fp32, the G query heads as the M side, tokens as
 // N), and reduces each head's logits over the block inside the warp: the
 // block's log-mass m + log(sum exp(z - m)) goes to `mass` as scratch. No CTA
@@ -33,14 +33,18 @@ constexpr float kLn2F = 0.69314718055994530942f;
 
 template <int D, int BLK>
 struct MassCfg {
-    static constexpr int kWarps = BLK == 64 ? 4 : 2;    // warps per CTA (shared memory bound)
+    static constexpr int kSub = 64;                      // tokens per staged tile (a block is BLK / 64 tiles)
+    static constexpr int kNSub = BLK / kSub;
+    static constexpr int kWarps = 4;
     static constexpr int kRowBytes = D * 2 + 16;         // padded tile row: conflict-free ldmatrix
-    static constexpr int kBufBytes = BLK * kRowBytes;    // one K tile
-    static constexpr int kSmem = kWarps * 2 * kBufBytes;  // two buffers per warp
-    static constexpr int kBlocksPerWarp = 4;
+    static constexpr int kBufBytes = kSub * kRowBytes;   // one staged tile
+    static constexpr int kStages = 3;                    // per warp: two tiles in flight, one computed
+    static constexpr int kSmem = kWarps * kStages * kBufBytes;
+    static constexpr int kBlocksPerWarp = 16 / kNSub;    // 16 tiles per warp
     static constexpr int kBlocksPerCta = kWarps * kBlocksPerWarp;
+    static constexpr int kTiles = kBlocksPerWarp * kNSub;
     static constexpr int kKSteps = D / 16;
-    static constexpr int kNT8 = BLK / 8;                 // n8 token tiles per block
+    static constexpr int kNT8 = kSub / 8;                // n8 token tiles per staged tile
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -52,12 +56,12 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Copies the K tile of block j (its valid rows only) into buffer `dst` (one warp).
+// Copies the valid rows of the 64 tokens starting at token t0 into buffer `dst` (one warp).
 template <int D, int BLK>
-__device__ __forceinline__ void load_tile(uint32_t dst, const __nv_bfloat16* krow, int j, int L, int lane) {
+__device__ __forceinline__ void load_tile(uint32_t dst, const __nv_bfloat16* krow, int t0, int L, int lane) {
     using C = MassCfg<D, BLK>;
-    const int nrows = min(BLK, L - j * BLK);
-    const __nv_bfloat16* src = krow + (size_t)j * BLK * D;
+    const int nrows = min(C::kSub, L - t0);
+    const __nv_bfloat16* src = krow + (size_t)t0 * D;
     constexpr int kPerRow = D * 2 / 16;
     for (int c = lane; c < nrows * kPerRow; c += 32) {
         const int r = c / kPerRow, q = c - r * kPerRow;
@@ -79,10 +83,13 @@ __global__ void __launch_bounds__(MassCfg<D, BLK>::kWarps * 32)
     const int G = Hq / Hkv;
     const int L = clamp_len(seq_lens[b], Lmax);
     const int NB = (L + BLK - 1) / BLK;
-    const int j0 = blockIdx.x * C::kBlocksPerCta + warp;  // this warp: j0, j0 + kWarps, ...
+    const int j0 = blockIdx.x * C::kBlocksPerCta + warp;  // this warp: blocks j0, j0 + kWarps, ...
     if (j0 >= NB) return;
     const __nv_bfloat16* krow = k_cache + (size_t)row * Lmax * D;
-    const uint32_t buf0 = smem_addr(smem) + warp * 2 * C::kBufBytes;
+    const uint32_t buf0 = smem_addr(smem) + warp * C::kStages * C::kBufBytes;
+    // the warp's staged tile u is half u % kNSub of its block u / kNSub
+    auto tile_t0 = [&](int u) { return (j0 + (u / C::kNSub) * C::kWarps) * BLK + (u % C::kNSub) * C::kSub; };
+    const int ntiles = min(C::kTiles, ((NB - 1 - j0) / C::kWarps + 1) * C::kNSub);
 
     // query fragments of the group's heads (rows g < G of the M = 16 side)
     uint32_t qa[C::kKSteps][2];
@@ -93,18 +100,20 @@ __global__ void __launch_bounds__(MassCfg<D, BLK>::kWarps * 32)
         qa[kk][1] = g < G ? *reinterpret_cast<const uint32_t*>(qh + kk * 16 + 8 + 2 * tig) : 0u;
     }
 
-    load_tile<D, BLK>(buf0, krow, j0, L, lane);
-    cp_async_commit();
-    int it = 0;
-    for (int j = j0, n = 0; n < C::kBlocksPerWarp && j < NB; j += C::kWarps, ++n, ++it) {
-        const int jn = j + C::kWarps;
-        const uint32_t cur = buf0 + (it & 1) * C::kBufBytes;
-        if (n + 1 < C::kBlocksPerWarp && jn < NB)
-            load_tile<D, BLK>(buf0 + ((it + 1) & 1) * C::kBufBytes, krow, jn, L, lane);
-        cp_async_commit();  // possibly empty: keeps one group per step
-        cp_async_wait<1>();
+    // stage s of the warp's ring holds its tiles u = s, s + 3, ...; one commit group per tile
+    for (int u = 0; u < C::kStages - 1; ++u) {
+        if (u < ntiles) load_tile<D, BLK>(buf0 + u * C::kBufBytes, krow, tile_t0(u), L, lane);
+        cp_async_commit();
+    }
+    float M = -INFINITY, S = 0.f;  // the current block's running max and sum (log2 domain)
+    for (int u = 0; u < ntiles; ++u) {
+        const int ua = u + C::kStages - 1;  // tile issued now
+        if (ua < ntiles) load_tile<D, BLK>(buf0 + (ua % C::kStages) * C::kBufBytes, krow, tile_t0(ua), L, lane);
+        cp_async_commit();  // possibly empty: keeps one group per tile
+        cp_async_wait<C::kStages - 1>();
         __syncwarp();
-        const int valid = min(BLK, L - j * BLK);
+        const uint32_t cur = buf0 + (u % C::kStages) * C::kBufBytes;
+        const int valid = min(C::kSub, L - tile_t0(u));  // <= 0: the empty half of a partial block
         float x[C::kNT8][2];
 #pragma unroll
         for (int nt = 0; nt < C::kNT8; ++nt) {
@@ -132,14 +141,23 @@ __global__ void __launch_bounds__(MassCfg<D, BLK>::kWarps * 32)
         for (int nt = 0; nt < C::kNT8; ++nt) m = fmaxf(m, fmaxf(x[nt][0], x[nt][1]));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        float sum = 0.f;
+        const float Mn = fmaxf(M, m);
+        if (Mn != -INFINITY) {
+            float sum = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < C::kNT8; ++nt) sum += exp2f(x[nt][0] - m) + exp2f(x[nt][1] - m);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (tig == 0 && g < G)
-            blse[((size_t)b * Hq + (size_t)kvh * G + g) * NBmax + j] = (m + log2f(sum)) * kLn2F;
-        __syncwarp();  // the buffer is refilled two steps later
+            for (int nt = 0; nt < C::kNT8; ++nt) sum += exp2f(x[nt][0] - Mn) + exp2f(x[nt][1] - Mn);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            S = S * exp2f(M - Mn) + sum;  // M = -inf: S is 0 and the factor is 0
+            M = Mn;
+        }
+        if (u % C::kNSub == C::kNSub - 1) {  // the block's last tile: write its log-mass
+            const int j = j0 + (u / C::kNSub) * C::kWarps;
+            if (tig == 0 && g < G) blse[((size_t)b * Hq + (size_t)kvh * G + g) * NBmax + j] = (M + log2f(S)) * kLn2F;
+            M = -INFINITY;
+            S = 0.f;
+        }
+        __syncwarp();  // the stage is refilled on the next step
     }
     cp_async_wait<0>();
 }
