@@ -56,8 +56,10 @@ def _load():
                                       ctypes.c_double, P, P]
         lib.oracle_merge.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, P, P]
         lib.oracle_block_mass.argtypes = [ctypes.POINTER(_Dims), P, P, P, ctypes.c_double, P, P]
+        lib.oracle_gate_scores_agg.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, ctypes.c_int32, P]
+        lib.oracle_select_threshold.argtypes = [ctypes.POINTER(_Dims), P, P, ctypes.c_int32, ctypes.c_double, P, P]
         for f in ("oracle_pool_project", "oracle_gate_scores", "oracle_select", "oracle_attend",
-                  "oracle_merge", "oracle_block_mass"):
+                  "oracle_merge", "oracle_block_mass", "oracle_gate_scores_agg", "oracle_select_threshold"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -135,6 +137,42 @@ def select_blocks(scores, seq_lens, block_size, max_seq_len, budget_tokens):
     dm = _dims(B, Hkv, Hkv, 0, 0, block_size, max_seq_len)
     _load().oracle_select(ctypes.byref(dm), sp, slp, int(budget_tokens),
                           idx.ctypes.data_as(ctypes.c_void_p), nsel.ctypes.data_as(ctypes.c_void_p))
+    return idx, nsel
+
+
+AGG_MEAN, AGG_MAX, AGG_SOFTMAX_MEAN = 0, 1, 2
+
+
+def gate_scores_agg(q_bits, w_q, kpool, seq_lens, block_size, max_seq_len, aggregation):
+    """Block scores with every head scored on its own, then aggregated over the group:
+    0 mean, 1 max, 2 mean of each head's softmax over its row's blocks. NaN past NB_b."""
+    q_bits, qp = _c(q_bits, np.uint16)
+    B, Hq, D = q_bits.shape
+    w_q, wp = _c(w_q, np.float32)
+    Hkv, dg = w_q.shape[0], w_q.shape[1]
+    kpool, kpp = _c(kpool, np.float64)
+    sl, slp = _c(seq_lens, np.int32)
+    NBmax = num_blocks(max_seq_len, block_size)
+    assert kpool.shape == (B, Hkv, NBmax, dg)
+    out = np.empty((B, Hkv, NBmax), np.float64)
+    dm = _dims(B, Hq, Hkv, D, dg, block_size, max_seq_len)
+    _load().oracle_gate_scores_agg(ctypes.byref(dm), qp, wp, kpp, slp, int(aggregation),
+                                   out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def select_threshold(scores, seq_lens, block_size, max_seq_len, budget_tokens, threshold):
+    """The last block plus the candidates scoring >= threshold, at most k_b-1 (the highest)."""
+    scores, sp = _c(scores, np.float64)
+    B, Hkv, NBmax = scores.shape
+    assert NBmax == num_blocks(max_seq_len, block_size)
+    sl, slp = _c(seq_lens, np.int32)
+    kmax = int(budget_tokens) // block_size
+    idx = np.empty((B, Hkv, kmax), np.int32)
+    nsel = np.empty((B, Hkv), np.int32)
+    dm = _dims(B, Hkv, Hkv, 0, 0, block_size, max_seq_len)
+    _load().oracle_select_threshold(ctypes.byref(dm), sp, slp, int(budget_tokens), float(threshold),
+                                    idx.ctypes.data_as(ctypes.c_void_p), nsel.ctypes.data_as(ctypes.c_void_p))
     return idx, nsel
 
 

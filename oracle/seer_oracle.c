@@ -344,3 +344,95 @@ void oracle_block_mass(const oracle_dims* dm, const uint16_t* q, const uint16_t*
         free(z);
     }
 }
+
+/* Gate variants (neither is on the pages; these are the readings taken).
+ * Aggregation of the G per-head scores of a group, every head scored
+ * explicitly (no use of linearity):
+ *   s_h[j] = (W_q[kvh] q_h) . kpool[b,kvh,j] / sqrt(dg),  j < NB_b
+ *   agg 0: s[j] = (1/G) sum_h s_h[j]                        (the mean gate)
+ *   agg 1: s[j] = max_h s_h[j]
+ *   agg 2: s[j] = (1/G) sum_h exp(s_h[j]) / sum_{i < NB_b} exp(s_h[i])
+ *          (each head's softmax over all of its row's blocks, then the mean)
+ * Entries j >= NB_b are NaN. */
+void oracle_gate_scores_agg(const oracle_dims* dm, const uint16_t* q, const float* w_q,
+                            const double* kpool, const int32_t* seq_lens, int32_t agg, double* scores) {
+    const int B = dm->batch, Hq = dm->num_q_heads, Hkv = dm->num_kv_heads;
+    const int D = dm->head_dim, dg = dm->gate_dim, blk = dm->block_size;
+    const int NBmax = num_blocks(dm->max_seq_len, blk);
+    const int G = Hq / Hkv;
+    const double inv_sqrt_dg = 1.0 / sqrt((double)dg);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int row = 0; row < B * Hkv; ++row) {
+        const int b = row / Hkv, kvh = row % Hkv;
+        const int NB = num_blocks(seq_lens[b], blk);
+        const float* W = w_q + (size_t)kvh * dg * D;
+        double* qg = (double*)malloc(sizeof(double) * (size_t)G * dg);
+        double* sh = (double*)malloc(sizeof(double) * (size_t)G * (NB > 0 ? NB : 1));
+        for (int h = 0; h < G; ++h) {
+            const uint16_t* qh = q + ((size_t)b * Hq + (size_t)kvh * G + h) * D;
+            for (int e = 0; e < dg; ++e) {
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += bf16_to_double(qh[d]) * (double)W[(size_t)e * D + d];
+                qg[(size_t)h * dg + e] = acc;
+            }
+            for (int j = 0; j < NB; ++j) {
+                const double* kp = kpool + (size_t)row * NBmax * dg + (size_t)j * dg;
+                double acc = 0.0;
+                for (int e = 0; e < dg; ++e) acc += qg[(size_t)h * dg + e] * kp[e];
+                sh[(size_t)h * NB + j] = acc * inv_sqrt_dg;
+            }
+            if (agg == 2 && NB > 0) {  /* this head's softmax over its row's blocks */
+                double m = -INFINITY, den = 0.0;
+                for (int j = 0; j < NB; ++j) if (sh[(size_t)h * NB + j] > m) m = sh[(size_t)h * NB + j];
+                for (int j = 0; j < NB; ++j) den += exp(sh[(size_t)h * NB + j] - m);
+                for (int j = 0; j < NB; ++j) sh[(size_t)h * NB + j] = exp(sh[(size_t)h * NB + j] - m) / den;
+            }
+        }
+        double* out = scores + (size_t)row * NBmax;
+        for (int j = 0; j < NBmax; ++j) out[j] = NAN;
+        for (int j = 0; j < NB; ++j) {
+            double a = (agg == 1) ? -INFINITY : 0.0;
+            for (int h = 0; h < G; ++h) {
+                const double v = sh[(size_t)h * NB + j];
+                if (agg == 1) a = v > a ? v : a;
+                else a += v;
+            }
+            out[j] = (agg == 1) ? a : a / (double)G;
+        }
+        free(qg);
+        free(sh);
+    }
+}
+
+/* Threshold selection (a reading; the pages describe a token budget only):
+ * block NB_b-1 always, plus the candidates 0 .. NB_b-2 whose score is at
+ * least `threshold`, at most k_b - 1 of them (the highest, equal scores to the
+ * lower index), ascending; -1 fills the rest of the kmax slots. */
+void oracle_select_threshold(const oracle_dims* dm, const double* scores, const int32_t* seq_lens,
+                             int32_t budget_tokens, double threshold, int32_t* block_idx,
+                             int32_t* num_selected) {
+    const int B = dm->batch, Hkv = dm->num_kv_heads, blk = dm->block_size;
+    const int NBmax = num_blocks(dm->max_seq_len, blk);
+    const int kmax = budget_tokens / blk;
+    for (int row = 0; row < B * Hkv; ++row) {
+        const int b = row / Hkv;
+        const int NB = num_blocks(seq_lens[b], blk);
+        const double* s = scores + (size_t)row * NBmax;
+        int32_t* out = block_idx + (size_t)row * kmax;
+        for (int i = 0; i < kmax; ++i) out[i] = -1;
+        if (NB == 0) { num_selected[row] = 0; continue; }
+        const int kb = kmax < NB ? kmax : NB;
+        scored_block* cand = (scored_block*)malloc(sizeof(scored_block) * (size_t)NB);
+        int nc = 0;
+        for (int j = 0; j < NB - 1; ++j)
+            if (s[j] >= threshold) { cand[nc].score = s[j]; cand[nc].index = j; ++nc; }
+        qsort(cand, (size_t)nc, sizeof(scored_block), by_score_then_index);
+        const int take = nc < kb - 1 ? nc : kb - 1;
+        int n = 0;
+        for (int i = 0; i < take; ++i) out[n++] = cand[i].index;
+        qsort(out, (size_t)n, sizeof(int32_t), ascending_int);
+        out[n] = NB - 1;
+        num_selected[row] = n + 1;
+        free(cand);
+    }
+}

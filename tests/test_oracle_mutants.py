@@ -45,6 +45,11 @@ MUTANTS = {
     "block_mass_ignores_length": [("L = L < 0 ? 0 : (L > Lmax ? Lmax : L);\n        double* z",
                                    "L = Lmax;\n        double* z")],
     "block_mass_lse_missing_max": [("const double lse_h = m + log(denom);", "const double lse_h = log(denom);")],
+    "agg_max_takes_min": [("if (agg == 1) a = v > a ? v : a;", "if (agg == 1) a = v < a ? v : a;")],
+    "agg_softmax_over_candidates_only": [("for (int j = 0; j < NB; ++j) den += exp(sh[(size_t)h * NB + j] - m);",
+                                          "for (int j = 0; j < NB - 1; ++j) den += exp(sh[(size_t)h * NB + j] - m);")],
+    "agg_mean_not_divided": [("out[j] = (agg == 1) ? a : a / (double)G;", "out[j] = a;")],
+    "threshold_strict": [("if (s[j] >= threshold)", "if (s[j] > threshold)")],
     "value_row_of_wrong_head": [("const uint16_t* vt = v_cache + ((size_t)row * Lmax + tok[i]) * D;",
                                  "const uint16_t* vt = v_cache + ((size_t)(row ^ 1) * Lmax + tok[i]) * D;")],
 }

@@ -403,3 +403,80 @@ def test_block_mass_single_block_and_empty(oracle):
     mass, lse = oracle.block_mass(c["q"], c["k"], c["lens"], wl.block_size)
     assert np.all(np.abs(mass[0, :, 0] - 1.0) < 1e-13) and np.all(mass[0, :, 1:] == 0.0)
     assert np.all(mass[1] == 0.0) and np.all(lse[1] == -np.inf)
+
+
+# ---------------------------------------------------------------- gate variants
+
+def _per_head_scores_torch(wl, c, kp):
+    # every head's score with torch float64 matmuls: (W_q q_h) . kpool_j / sqrt(dg)
+    q = torch.from_numpy(widen(c["q"]))
+    Wq = torch.from_numpy(c["w_q"].astype(np.float64))
+    KP = torch.from_numpy(kp)
+    G = wl.group
+    out = torch.full((wl.batch, wl.num_q_heads, wl.nb_max), float("nan"), dtype=torch.float64)
+    for b in range(wl.batch):
+        NB = -(-int(c["lens"][b]) // wl.block_size)
+        for h in range(wl.num_q_heads):
+            qg = Wq[h // G] @ q[b, h]
+            out[b, h, :NB] = (KP[b, h // G, :NB] @ qg) / math.sqrt(wl.gate_dim)
+    return out
+
+
+@pytest.mark.parametrize("agg", [0, 1, 2])
+def test_gate_aggregations_match_torch(oracle, agg):
+    for seed, dg in ((0, 64), (1, 32)):
+        wl, c = small_case(seed, dg=dg, lens=(320, 150))
+        kp = oracle.pool_project(c["k"], c["w_k"], c["lens"], wl.block_size)
+        got = oracle.gate_scores_agg(c["q"], c["w_q"], kp, c["lens"], wl.block_size, wl.max_seq_len, agg)
+        sh = _per_head_scores_torch(wl, c, kp)
+        G = wl.group
+        for b in range(wl.batch):
+            NB = -(-int(c["lens"][b]) // wl.block_size)
+            for kvh in range(wl.num_kv_heads):
+                grp = sh[b, kvh * G:(kvh + 1) * G, :NB]
+                ref = {0: grp.mean(0), 1: grp.max(0).values, 2: torch.softmax(grp, 1).mean(0)}[agg]
+                np.testing.assert_allclose(got[b, kvh, :NB], ref.numpy(), rtol=1e-12, atol=1e-15)
+                assert np.all(np.isnan(got[b, kvh, NB:]))
+                if agg == 2:
+                    assert abs(got[b, kvh, :NB].sum() - 1.0) < 1e-12
+
+
+def test_gate_aggregations_agree_when_heads_agree(oracle):
+    # identical query heads: max = mean, and the softmax-mean is the softmax of the mean gate
+    wl, c = small_case(2)
+    G = wl.group
+    for b in range(wl.batch):
+        for kvh in range(wl.num_kv_heads):
+            c["q"][b, kvh * G:(kvh + 1) * G] = c["q"][b, kvh * G]
+    kp = oracle.pool_project(c["k"], c["w_k"], c["lens"], wl.block_size)
+    mean = oracle.gate_scores_agg(c["q"], c["w_q"], kp, c["lens"], wl.block_size, wl.max_seq_len, 0)
+    mx = oracle.gate_scores_agg(c["q"], c["w_q"], kp, c["lens"], wl.block_size, wl.max_seq_len, 1)
+    sm = oracle.gate_scores_agg(c["q"], c["w_q"], kp, c["lens"], wl.block_size, wl.max_seq_len, 2)
+    np.testing.assert_allclose(mx, mean, rtol=0, atol=1e-15)
+    for b in range(wl.batch):
+        NB = -(-int(c["lens"][b]) // wl.block_size)
+        for kvh in range(wl.num_kv_heads):
+            ref = torch.softmax(torch.from_numpy(mean[b, kvh, :NB]), 0).numpy()
+            np.testing.assert_allclose(sm[b, kvh, :NB], ref, rtol=1e-12, atol=0)
+
+
+def test_threshold_selection_brute_force(oracle):
+    rng = np.random.default_rng(8)
+    B, Hkv, blk, Lmax = 3, 2, 64, 64 * 40
+    lens = np.array([Lmax, 64 * 17 + 5, 64], np.int32)
+    scores = np.round(rng.standard_normal((B, Hkv, 40)), 1)  # many exact ties, some at the threshold
+    for budget, tau in ((64 * 8, 0.3), (64 * 8, -np.inf), (64 * 8, np.inf), (64 * 40, 0.0), (64 * 3, -0.5)):
+        idx, nsel = oracle.select_threshold(scores, lens, blk, Lmax, budget, tau)
+        kmax = budget // blk
+        for b in range(B):
+            NB = -(-int(lens[b]) // blk)
+            kb = min(kmax, NB)
+            for h in range(Hkv):
+                cand = [j for j in range(NB - 1) if scores[b, h, j] >= tau]
+                cand.sort(key=lambda j: (-scores[b, h, j], j))
+                ref = sorted(cand[:kb - 1]) + [NB - 1]
+                assert nsel[b, h] == len(ref)
+                assert list(idx[b, h, :len(ref)]) == ref and np.all(idx[b, h, len(ref):] == -1)
+    top_i, top_n = oracle.select_blocks(scores, lens, blk, Lmax, 64 * 8)
+    thr_i, thr_n = oracle.select_threshold(scores, lens, blk, Lmax, 64 * 8, -np.inf)
+    assert np.array_equal(top_i, thr_i) and np.array_equal(top_n, thr_n)
