@@ -60,6 +60,7 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--dense-steps", type=int, default=30, help="timed steps of the dense baseline (0: skip)")
     p.add_argument("--mass-steps", type=int, default=30, help="timed calls of the block-level ground truth (0: skip)")
+    p.add_argument("--variant-steps", type=int, default=30, help="timed calls of each gate variant (0: skip)")
     return p.parse_args()
 
 
@@ -456,6 +457,36 @@ def run_ours(args):
                       "bytes": mass_bytes, "gbs": round(mass_bytes / (mass_us * 1e-6) / 1e9, 1),
                       "frac": round(mass_bytes / (mass_us * 1e-6) / 1e9 / peak, 4)}
 
+    # ---- gate variants: per-head aggregations of the block scores and threshold selection
+    variants = None
+    if args.variant_steps > 0:
+        def timed(fn):
+            v_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.variant_steps)]
+            for k in range(args.variant_steps + 3):
+                prepare()
+                evs = v_ev[k - 3] if k >= 3 else None
+                if evs:
+                    evs[0].record(stream)
+                fn()
+                if evs:
+                    evs[1].record(stream)
+            torch.cuda.synchronize()
+            us = float(np.mean([e[0].elapsed_time(e[1]) for e in v_ev])) * 1e3
+            return max_over_ranks([us], dev)[0] if world > 1 else us
+        nb_rows = [-(-min(int(L), wl.max_seq_len) // wl.block_size) for L in lens]
+        kp_bytes = sum(nb_rows) * wl.num_kv_heads * wl.gate_dim * 4  # one scan of every row's pooled keys
+        vs = torch.empty_like(st.scores)
+        variants = {"scan_bytes": kp_bytes}
+        for name, agg in (("mean", api.AGG_MEAN), ("max", api.AGG_MAX), ("softmax_mean", api.AGG_SOFTMAX_MEAN)):
+            us = timed(lambda: api.seer_gate_scores_agg(st.dims, inp["q"], inp["w_q"], st.kpool, inp["seq_lens"],
+                                                        agg, vs))
+            variants[f"agg_{name}_us"] = round(us, 3)
+            variants[f"agg_{name}_frac"] = round(kp_bytes / (us * 1e-6) / 1e9 / peak, 4)
+        thr_idx = torch.empty_like(st.block_idx)
+        thr_ns = torch.empty_like(st.num_selected)
+        variants["threshold_select_us"] = round(timed(lambda: api.seer_select_blocks_threshold(
+            st.dims, vs, inp["seq_lens"], st.budget_tokens, 0.0, thr_idx, thr_ns)), 3)
+
     # ---- end to end through the public API: host inputs in, host output out, every step.
     # The step's inputs (q and the new token's K/V rows) travel as one packed pinned buffer;
     # seer_append_kv places the token in the caches, the fused step runs, out comes back.
@@ -523,6 +554,7 @@ def run_ours(args):
             "separate_calls": separate,
             "dense_baseline": dense,
             "block_mass": block_mass,
+            "gate_variants": variants,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,

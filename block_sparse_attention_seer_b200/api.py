@@ -49,6 +49,8 @@ def _load_library():
         "seer_combine": [D, P, P, I32, P, P, P],
         "seer_append_kv": [D, P, P, P, P, P, P],
         "seer_block_mass": [D, P, P, P, F32, P, P, P],
+        "seer_gate_scores_agg": [D, P, P, P, P, I32, P, P],
+        "seer_select_blocks_threshold": [D, P, P, I32, F32, P, P, P],
         "seer_default_num_splits": [I32, P],
         "seer_decode_wait_failures": [P, I32],
         "seer_decode_step_workspace_size": [D, I32, P],
@@ -136,6 +138,24 @@ def seer_sparse_decode(dims, q, k_cache, v_cache, seq_lens, block_idx, num_selec
 def seer_combine(dims, o_part, lse_part, num_splits, out, lse_out, stream=None):
     _check("seer_combine", LIB.seer_combine(ctypes.byref(dims), _ptr(o_part), _ptr(lse_part), int(num_splits),
                                             _ptr(out), _ptr(lse_out), _stream(stream)))
+
+
+AGG_MEAN, AGG_MAX, AGG_SOFTMAX_MEAN = 0, 1, 2
+
+
+def seer_gate_scores_agg(dims, q, w_q, kpool, seq_lens, aggregation, scores, stream=None):
+    """Per-head block scores aggregated over the group: AGG_MEAN, AGG_MAX or AGG_SOFTMAX_MEAN."""
+    _check("seer_gate_scores_agg", LIB.seer_gate_scores_agg(ctypes.byref(dims), _ptr(q), _ptr(w_q), _ptr(kpool),
+                                                            _ptr(seq_lens), int(aggregation), _ptr(scores),
+                                                            _stream(stream)))
+
+
+def seer_select_blocks_threshold(dims, scores, seq_lens, budget_tokens, threshold, block_idx, num_selected,
+                                 stream=None):
+    """The last block plus at most k_b-1 candidates scoring >= threshold (the highest), ascending."""
+    _check("seer_select_blocks_threshold",
+           LIB.seer_select_blocks_threshold(ctypes.byref(dims), _ptr(scores), _ptr(seq_lens), int(budget_tokens),
+                                            float(threshold), _ptr(block_idx), _ptr(num_selected), _stream(stream)))
 
 
 def seer_block_mass(dims, q, k_cache, seq_lens, mass, lse_out=None, sm_scale=0.0, stream=None):

@@ -180,6 +180,32 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
     return from_cuda(seer::launch_combine(s, o_part, lse_part, num_splits, out, lse_out, stream));
 }
 
+seer_status seer_gate_scores_agg(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
+                                 const int32_t* seq_lens, int32_t aggregation, float* scores, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !w_q || !kpool || !seq_lens || !scores) return SEER_ERR_INVALID_ARG;
+    if (aggregation < SEER_AGG_MEAN || aggregation > SEER_AGG_SOFTMAX_MEAN) return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(w_q, 16) || !aligned(kpool, 16)) return SEER_ERR_INVALID_ARG;
+    return from_cuda(seer::launch_gate_scores_agg(s, q, w_q, kpool, seq_lens, aggregation, scores, stream));
+}
+
+seer_status seer_select_blocks_threshold(const seer_dims* dims, const float* scores, const int32_t* seq_lens,
+                                         int32_t budget_tokens, float threshold, int32_t* block_idx,
+                                         int32_t* num_selected, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!scores || !seq_lens || !block_idx || !num_selected) return SEER_ERR_INVALID_ARG;
+    if (budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
+    if (threshold != threshold) return SEER_ERR_INVALID_ARG;  // NaN: no order against it
+    if (s.NBmax > 16384) return SEER_ERR_UNSUPPORTED;
+    return from_cuda(
+        seer::launch_select_threshold(s, scores, seq_lens, budget_tokens / s.blk, threshold, block_idx, num_selected,
+                                      stream));
+}
+
 seer_status seer_block_mass(const seer_dims* dims, const void* q, const void* k_cache, const int32_t* seq_lens,
                             float sm_scale, float* mass, float* lse_out, cudaStream_t stream) {
     Shape s;

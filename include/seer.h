@@ -188,6 +188,31 @@ seer_status seer_sparse_decode(const seer_dims* dims, const void* q, const void*
 seer_status seer_combine(const seer_dims* dims, const float* o_part, const float* lse_part,
                          int32_t num_splits, void* out, float* lse_out, cudaStream_t stream);
 
+/* Gate variants. Neither page says how the G query heads of a GQA group share
+ * one block score, nor whether a threshold may replace the token budget; the
+ * mean gate and top-k above are the plain readings, these are the
+ * alternatives (every head scored on its own first):
+ *   s_h[j] = (W_q q_h) . kpool[b, kvh, j] / sqrt(dg)
+ *   SEER_AGG_MEAN          s[j] = (1/G) sum_h s_h[j]   (same as seer_gate_scores up to rounding)
+ *   SEER_AGG_MAX           s[j] = max_h s_h[j]
+ *   SEER_AGG_SOFTMAX_MEAN  s[j] = (1/G) sum_h exp(s_h[j]) / sum_{i < NB_b} exp(s_h[i])
+ * Arguments, layouts and errors as seer_gate_scores; an aggregation outside
+ * the three values is SEER_ERR_INVALID_ARG.
+ *
+ * seer_select_blocks_threshold keeps block NB_b - 1 plus the candidates
+ * 0 .. NB_b - 2 whose score is >= threshold, at most k_b - 1 of them (the
+ * highest; equal scores to the lower index), ascending; num_selected = their
+ * count + 1 (0 for an empty sequence); -1 fills the rest of the kmax slots.
+ * threshold = -inf gives seer_select_blocks. Arguments as seer_select_blocks;
+ * a NaN threshold is SEER_ERR_INVALID_ARG.
+ */
+enum { SEER_AGG_MEAN = 0, SEER_AGG_MAX = 1, SEER_AGG_SOFTMAX_MEAN = 2 };
+seer_status seer_gate_scores_agg(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
+                                 const int32_t* seq_lens, int32_t aggregation, float* scores, cudaStream_t stream);
+seer_status seer_select_blocks_threshold(const seer_dims* dims, const float* scores, const int32_t* seq_lens,
+                                         int32_t budget_tokens, float threshold, int32_t* block_idx,
+                                         int32_t* num_selected, cudaStream_t stream);
+
 /* Block-level ground truth of one decode query. "SeerAttention: Learning
  * Intrinsic Sparse Attention in Your LLMs" (abstract) distils its gate from a
  * block-level ground truth extracted by a customised attention kernel; read

@@ -84,6 +84,23 @@ def test_null_pointers_and_bad_scalars_rejected():
     assert L.seer_default_num_splits(0, ctypes.byref(ctypes.c_int32())) == api.SEER_ERR_INVALID_ARG
 
 
+def test_gate_variants_validate_on_host():
+    d = _dims()
+    L = api.LIB
+    assert L.seer_gate_scores_agg(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 3, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_gate_scores_agg(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, -1, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_gate_scores_agg(ctypes.byref(d), None, FAKE, FAKE, FAKE, 0, FAKE, None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_select_blocks_threshold(ctypes.byref(d), FAKE, FAKE, 64, float("nan"), FAKE, FAKE,
+                                          None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_select_blocks_threshold(ctypes.byref(d), FAKE, FAKE, 100, 0.0, FAKE, FAKE,
+                                          None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_select_blocks_threshold(ctypes.byref(d), FAKE, FAKE, 64, 0.0, None, FAKE,
+                                          None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_block_mass(ctypes.byref(d), FAKE, FAKE, FAKE, float("inf"), FAKE, None,
+                             None) == api.SEER_ERR_INVALID_ARG
+    assert L.seer_block_mass(ctypes.byref(d), FAKE, FAKE, FAKE, 0.0, None, None, None) == api.SEER_ERR_INVALID_ARG
+
+
 def test_append_kv_validates_on_host():
     d = _dims()
     L = api.LIB
