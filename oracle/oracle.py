@@ -58,8 +58,13 @@ def _load():
         lib.oracle_block_mass.argtypes = [ctypes.POINTER(_Dims), P, P, P, ctypes.c_double, P, P]
         lib.oracle_gate_scores_agg.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, ctypes.c_int32, P]
         lib.oracle_select_threshold.argtypes = [ctypes.POINTER(_Dims), P, P, ctypes.c_int32, ctypes.c_double, P, P]
+        lib.oracle_prefill_gate.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P]
+        lib.oracle_prefill_select.argtypes = [ctypes.POINTER(_Dims), P, P, ctypes.c_int32, P, P]
+        lib.oracle_prefill_attend.argtypes = [ctypes.POINTER(_Dims), P, P, P, P, P, P, ctypes.c_int32,
+                                              ctypes.c_double, P, P]
         for f in ("oracle_pool_project", "oracle_gate_scores", "oracle_select", "oracle_attend",
-                  "oracle_merge", "oracle_block_mass", "oracle_gate_scores_agg", "oracle_select_threshold"):
+                  "oracle_merge", "oracle_block_mass", "oracle_gate_scores_agg", "oracle_select_threshold",
+                  "oracle_prefill_gate", "oracle_prefill_select", "oracle_prefill_attend"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -174,6 +179,64 @@ def select_threshold(scores, seq_lens, block_size, max_seq_len, budget_tokens, t
     _load().oracle_select_threshold(ctypes.byref(dm), sp, slp, int(budget_tokens), float(threshold),
                                     idx.ctypes.data_as(ctypes.c_void_p), nsel.ctypes.data_as(ctypes.c_void_p))
     return idx, nsel
+
+
+def prefill_gate(q_bits, w_q, kpool, seq_lens, block_size):
+    """Prefill block scores s[b, kvh, i, j] (query block i, key block j <= i); NaN elsewhere.
+
+    q_bits uint16 [B, Hq, Lmax, D]; w_q float32 [Hkv, dg, D]; kpool float64 [B, Hkv, NBmax, dg].
+    """
+    q_bits, qp = _c(q_bits, np.uint16)
+    B, Hq, Lmax, D = q_bits.shape
+    w_q, wp = _c(w_q, np.float32)
+    Hkv, dg = w_q.shape[0], w_q.shape[1]
+    kpool, kpp = _c(kpool, np.float64)
+    sl, slp = _c(seq_lens, np.int32)
+    nbm = num_blocks(Lmax, block_size)
+    out = np.empty((B, Hkv, nbm, nbm), np.float64)
+    dm = _dims(B, Hq, Hkv, D, dg, block_size, Lmax)
+    _load().oracle_prefill_gate(ctypes.byref(dm), qp, wp, kpp, slp, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def prefill_select(scores, seq_lens, block_size, max_seq_len, budget_tokens):
+    """Per query block i: block i plus the top min(k, i+1)-1 of blocks < i, ascending.
+
+    Returns (block_idx int32 [B, Hkv, NBmax, kmax] -1 padded, num_selected int32 [B, Hkv, NBmax]).
+    """
+    scores, sp = _c(scores, np.float64)
+    B, Hkv, nbm, _ = scores.shape
+    sl, slp = _c(seq_lens, np.int32)
+    kmax = int(budget_tokens) // block_size
+    idx = np.empty((B, Hkv, nbm, kmax), np.int32)
+    nsel = np.empty((B, Hkv, nbm), np.int32)
+    dm = _dims(B, Hkv, Hkv, 0, 0, block_size, max_seq_len)
+    _load().oracle_prefill_select(ctypes.byref(dm), sp, slp, int(budget_tokens), idx.ctypes.data_as(ctypes.c_void_p),
+                                  nsel.ctypes.data_as(ctypes.c_void_p))
+    return idx, nsel
+
+
+def prefill_attend(q_bits, k_bits, v_bits, seq_lens, block_idx, num_selected, block_size, sm_scale=0.0):
+    """Causal attention of every prompt token over the kept blocks of its query block.
+
+    q_bits uint16 [B, Hq, Lmax, D]; k/v uint16 [B, Hkv, Lmax, D]; block_idx [B, Hkv, NBmax, kmax].
+    Returns (out float64 [B, Hq, Lmax, D], lse float64 [B, Hq, Lmax]); rows past L_b are 0 / -inf.
+    """
+    q_bits, qp = _c(q_bits, np.uint16)
+    k_bits, kp_ = _c(k_bits, np.uint16)
+    v_bits, vp = _c(v_bits, np.uint16)
+    B, Hq, Lmax, D = q_bits.shape
+    Hkv = k_bits.shape[1]
+    sl, slp = _c(seq_lens, np.int32)
+    block_idx, ip = _c(block_idx, np.int32)
+    num_selected, np_ = _c(num_selected, np.int32)
+    kmax = block_idx.shape[-1]
+    out = np.empty((B, Hq, Lmax, D), np.float64)
+    lse = np.empty((B, Hq, Lmax), np.float64)
+    dm = _dims(B, Hq, Hkv, D, 0, block_size, Lmax)
+    _load().oracle_prefill_attend(ctypes.byref(dm), qp, kp_, vp, slp, ip, np_, int(kmax), float(sm_scale),
+                                  out.ctypes.data_as(ctypes.c_void_p), lse.ctypes.data_as(ctypes.c_void_p))
+    return out, lse
 
 
 def attend(q_bits, k_bits, v_bits, seq_lens, block_idx, num_selected, block_size, sm_scale=0.0):

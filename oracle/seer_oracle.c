@@ -436,3 +436,148 @@ void oracle_select_threshold(const oracle_dims* dm, const double* scores, const 
         free(cand);
     }
 }
+
+/* ------------------------------------------------------------ block-sparse prefill
+ * [V1] (pool Q and K along the sequence, linear layers, multiply to block
+ * scores; a block-sparse attention over the kept blocks) read for a causal
+ * prompt of L_b tokens, with the decode gate's readings (mean pool over valid
+ * tokens, one bias-free map per KV head, mean over the group's heads, 1/sqrt(dg))
+ * and selection rule (the diagonal block plays the decode's last block).
+ * q: bf16 bits [B, Hq, Lmax, D]; query block i = tokens [i*blk, min((i+1)*blk, L_b)).
+ *
+ * Gate: qbar[h,i] = mean_{t in block i} q[b,h,t,:];  qg = W_q[kvh] qbar
+ *   s[b,kvh,i,j] = (1/G) sum_h qg[h,i] . kpool[b,kvh,j] / sqrt(dg)   j <= i < NB_b
+ * Entries with j > i or i >= NB_b are NaN. Shape [B, Hkv, NBmax, NBmax]. */
+void oracle_prefill_gate(const oracle_dims* dm, const uint16_t* q, const float* w_q, const double* kpool,
+                         const int32_t* seq_lens, double* scores) {
+    const int B = dm->batch, Hq = dm->num_q_heads, Hkv = dm->num_kv_heads;
+    const int D = dm->head_dim, dg = dm->gate_dim, blk = dm->block_size, Lmax = dm->max_seq_len;
+    const int NBmax = num_blocks(Lmax, blk);
+    const int G = Hq / Hkv;
+    const double inv_sqrt_dg = 1.0 / sqrt((double)dg);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int row = 0; row < B * Hkv; ++row) {
+        const int b = row / Hkv, kvh = row % Hkv;
+        const int L = seq_lens[b];
+        const int NB = num_blocks(L, blk);
+        const float* W = w_q + (size_t)kvh * dg * D;
+        double* qbar = (double*)malloc(sizeof(double) * (size_t)D);
+        double* qg = (double*)malloc(sizeof(double) * (size_t)dg);
+        double* out = scores + (size_t)row * NBmax * NBmax;
+        for (size_t x = 0; x < (size_t)NBmax * NBmax; ++x) out[x] = NAN;
+        for (int i = 0; i < NB; ++i) {
+            const int t0 = i * blk, t1 = (t0 + blk < L) ? t0 + blk : L;
+            for (int j = 0; j <= i; ++j) out[(size_t)i * NBmax + j] = 0.0;
+            for (int h = 0; h < G; ++h) {
+                const uint16_t* qh = q + ((size_t)b * Hq + (size_t)kvh * G + h) * Lmax * D;
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int t = t0; t < t1; ++t) acc += bf16_to_double(qh[(size_t)t * D + d]);
+                    qbar[d] = acc / (double)(t1 - t0);
+                }
+                for (int e = 0; e < dg; ++e) {
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += qbar[d] * (double)W[(size_t)e * D + d];
+                    qg[e] = acc;
+                }
+                for (int j = 0; j <= i; ++j) {
+                    const double* kp = kpool + (size_t)row * NBmax * dg + (size_t)j * dg;
+                    double acc = 0.0;
+                    for (int e = 0; e < dg; ++e) acc += qg[e] * kp[e];
+                    out[(size_t)i * NBmax + j] += acc * inv_sqrt_dg / (double)G;
+                }
+            }
+        }
+        free(qbar);
+        free(qg);
+    }
+}
+
+/* Selection of each query block i < NB_b: block i itself plus the top
+ * min(k, i + 1) - 1 of blocks 0 .. i-1 (higher score, then lower index),
+ * ascending; k = budget / blk. block_idx [B, Hkv, NBmax, kmax] (-1 padded),
+ * num_selected [B, Hkv, NBmax] (0 for i >= NB_b). */
+void oracle_prefill_select(const oracle_dims* dm, const double* scores, const int32_t* seq_lens,
+                           int32_t budget_tokens, int32_t* block_idx, int32_t* num_selected) {
+    const int B = dm->batch, Hkv = dm->num_kv_heads, blk = dm->block_size;
+    const int NBmax = num_blocks(dm->max_seq_len, blk);
+    const int kmax = budget_tokens / blk;
+    for (int row = 0; row < B * Hkv; ++row) {
+        const int NB = num_blocks(seq_lens[row / Hkv], blk);
+        for (int i = 0; i < NBmax; ++i) {
+            int32_t* out = block_idx + ((size_t)row * NBmax + i) * kmax;
+            for (int x = 0; x < kmax; ++x) out[x] = -1;
+            int32_t* ns = num_selected + (size_t)row * NBmax + i;
+            if (i >= NB) { *ns = 0; continue; }
+            const double* s = scores + ((size_t)row * NBmax + i) * NBmax;
+            const int ki = kmax < i + 1 ? kmax : i + 1;
+            scored_block* cand = (scored_block*)malloc(sizeof(scored_block) * (size_t)(i > 0 ? i : 1));
+            for (int j = 0; j < i; ++j) { cand[j].score = s[j]; cand[j].index = j; }
+            qsort(cand, (size_t)i, sizeof(scored_block), by_score_then_index);
+            int n = 0;
+            for (int x = 0; x < ki - 1; ++x) out[n++] = cand[x].index;
+            qsort(out, (size_t)n, sizeof(int32_t), ascending_int);
+            out[n] = i;
+            *ns = n + 1;
+            free(cand);
+        }
+    }
+}
+
+/* Causal block-sparse attention: query token t < L_b of query block i = t/blk
+ * and head h attends to the tokens u <= t (u < L_b) of the kept blocks of
+ * (b, kvh, i):  out = softmax(q_t . K_u * scale) V_u,  lse = log sum exp.
+ * Rows t >= L_b: out 0, lse -inf. out [B, Hq, Lmax, D], lse [B, Hq, Lmax].
+ * Indices outside [0, i] are skipped. sm_scale <= 0 means 1/sqrt(D). */
+void oracle_prefill_attend(const oracle_dims* dm, const uint16_t* q, const uint16_t* k_cache,
+                           const uint16_t* v_cache, const int32_t* seq_lens, const int32_t* block_idx,
+                           const int32_t* num_selected, int32_t kmax, double sm_scale, double* out, double* lse) {
+    const int B = dm->batch, Hq = dm->num_q_heads, Hkv = dm->num_kv_heads;
+    const int D = dm->head_dim, blk = dm->block_size, Lmax = dm->max_seq_len;
+    const int NBmax = num_blocks(Lmax, blk);
+    const int G = Hq / Hkv;
+    const double scale = (sm_scale > 0.0) ? sm_scale : 1.0 / sqrt((double)D);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * Hq; ++bh) {
+        const int b = bh / Hq, hq = bh % Hq, kvh = hq / G;
+        const int row = b * Hkv + kvh;
+        const int L = seq_lens[b];
+        double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        int32_t* tok = (int32_t*)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
+        for (int t = 0; t < Lmax; ++t) {
+            double* o = out + ((size_t)bh * Lmax + t) * D;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            if (t >= L) { lse[(size_t)bh * Lmax + t] = -INFINITY; continue; }
+            const int i = t / blk;
+            const int32_t* idx = block_idx + ((size_t)row * NBmax + i) * kmax;
+            const int nsel = num_selected[(size_t)row * NBmax + i];
+            int n = 0;
+            for (int x = 0; x < nsel; ++x) {
+                const int j = idx[x];
+                if (j < 0 || j > i) continue;
+                for (int u = j * blk; u < (j + 1) * blk && u <= t && u < L; ++u) tok[n++] = u;
+            }
+            const uint16_t* qt = q + ((size_t)bh * Lmax + t) * D;
+            double m = -INFINITY;
+            for (int x = 0; x < n; ++x) {
+                const uint16_t* ku = k_cache + ((size_t)row * Lmax + tok[x]) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += bf16_to_double(qt[d]) * bf16_to_double(ku[d]);
+                z[x] = acc * scale;
+                if (z[x] > m) m = z[x];
+            }
+            if (n == 0) { lse[(size_t)bh * Lmax + t] = -INFINITY; continue; }
+            double den = 0.0;
+            for (int x = 0; x < n; ++x) {
+                const double p = exp(z[x] - m);
+                den += p;
+                const uint16_t* vu = v_cache + ((size_t)row * Lmax + tok[x]) * D;
+                for (int d = 0; d < D; ++d) o[d] += p * bf16_to_double(vu[d]);
+            }
+            for (int d = 0; d < D; ++d) o[d] /= den;
+            lse[(size_t)bh * Lmax + t] = m + log(den);
+        }
+        free(z);
+        free(tok);
+    }
+}

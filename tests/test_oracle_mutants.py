@@ -50,6 +50,11 @@ MUTANTS = {
                                           "for (int j = 0; j < NB - 1; ++j) den += exp(sh[(size_t)h * NB + j] - m);")],
     "agg_mean_not_divided": [("out[j] = (agg == 1) ? a : a / (double)G;", "out[j] = a;")],
     "threshold_strict": [("if (s[j] >= threshold)", "if (s[j] > threshold)")],
+    "prefill_not_causal": [("for (int u = j * blk; u < (j + 1) * blk && u <= t && u < L; ++u) tok[n++] = u;",
+                            "for (int u = j * blk; u < (j + 1) * blk && u < L; ++u) tok[n++] = u;")],
+    "prefill_query_pool_summed": [("qbar[d] = acc / (double)(t1 - t0);", "qbar[d] = acc;")],
+    "prefill_diagonal_not_forced": [("            out[n] = i;\n            *ns = n + 1;",
+                                     "            out[n] = (i > 0 && n > 0) ? out[n - 1] : i;\n            *ns = n + 1;")],
     "value_row_of_wrong_head": [("const uint16_t* vt = v_cache + ((size_t)row * Lmax + tok[i]) * D;",
                                  "const uint16_t* vt = v_cache + ((size_t)(row ^ 1) * Lmax + tok[i]) * D;")],
 }

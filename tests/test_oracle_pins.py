@@ -480,3 +480,103 @@ def test_threshold_selection_brute_force(oracle):
     top_i, top_n = oracle.select_blocks(scores, lens, blk, Lmax, 64 * 8)
     thr_i, thr_n = oracle.select_threshold(scores, lens, blk, Lmax, 64 * 8, -np.inf)
     assert np.array_equal(top_i, thr_i) and np.array_equal(top_n, thr_n)
+
+
+# ---------------------------------------------------------------- block-sparse prefill
+
+def prefill_case(seed, B=2, Hq=4, Hkv=2, D=64, dg=64, blk=64, Lmax=320, lens=(320, 200)):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Hq, Lmax, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Lmax, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Lmax, D, generator=g).to(torch.bfloat16)
+    u16 = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    wq = (torch.randn(Hkv, dg, D, generator=g) / math.sqrt(D)).numpy()
+    wk = (torch.randn(Hkv, dg, D, generator=g) / math.sqrt(D)).numpy()
+    return dict(q=u16(q), k=u16(k), v=u16(v), w_q=wq, w_k=wk, lens=np.array(lens, np.int32), blk=blk, G=Hq // Hkv)
+
+
+def test_prefill_gate_identity_weights_closed_form(oracle):
+    # W = I: s[i, j] = mean_h(mean of q_h over block i) . mean(K over block j) / sqrt(D)
+    c = prefill_case(0)
+    D = c["q"].shape[-1]
+    eye = np.broadcast_to(np.eye(D, dtype=np.float32), (2, D, D)).copy()
+    kp = oracle.pool_project(c["k"], eye, c["lens"], c["blk"])
+    s = oracle.prefill_gate(c["q"], eye, kp, c["lens"], c["blk"])
+    Q, K = widen(c["q"]), widen(c["k"])
+    G, blk = c["G"], c["blk"]
+    for b, L in enumerate(int(x) for x in c["lens"]):
+        NB = -(-L // blk)
+        for kvh in range(2):
+            for i in range(NB):
+                qb = Q[b, kvh * G:(kvh + 1) * G, i * blk:min(i * blk + blk, L)].mean(1).mean(0)
+                for j in range(NB):
+                    kb = K[b, kvh, j * blk:min(j * blk + blk, L)].mean(0)
+                    if j <= i:
+                        assert abs(s[b, kvh, i, j] - qb @ kb / math.sqrt(D)) < 1e-12
+                    else:
+                        assert math.isnan(s[b, kvh, i, j])
+        assert np.all(np.isnan(s[b, :, NB:]))
+
+
+def test_prefill_selection_is_decode_selection_per_query_block(oracle):
+    c = prefill_case(1, Lmax=64 * 12, lens=(64 * 12, 64 * 7 + 3))
+    kp = oracle.pool_project(c["k"], c["w_k"], c["lens"], c["blk"])
+    s = oracle.prefill_gate(c["q"], c["w_q"], kp, c["lens"], c["blk"])
+    s = np.round(s, 3)  # ties
+    for budget in (64, 64 * 4, 64 * 20):
+        idx, ns = oracle.prefill_select(s, c["lens"], 64, 64 * 12, budget)
+        kmax = budget // 64
+        for b, L in enumerate(int(x) for x in c["lens"]):
+            NB = -(-L // 64)
+            for i in range(12):
+                if i >= NB:
+                    assert ns[b, :, i].tolist() == [0, 0] and np.all(idx[b, :, i] == -1)
+                    continue
+                # the decode rule on a sequence of i + 1 blocks whose scores are row i
+                row = np.full((2, 2, 12), np.nan)
+                row[0, :, :i + 1] = s[b, :, i, :i + 1]
+                r_idx, r_ns = oracle.select_blocks(row[:1], np.array([(i + 1) * 64], np.int32), 64, 64 * 12, budget)
+                assert ns[b, :, i].tolist() == r_ns[0].tolist()
+                assert np.array_equal(idx[b, :, i], r_idx[0]) and kmax == idx.shape[-1]
+
+
+def test_prefill_dense_equals_torch_causal_sdpa(oracle):
+    for blk in (64, 128):
+        c = prefill_case(2, blk=blk, Lmax=256, lens=(256, 190))
+        nbm = 256 // blk
+        idx = np.full((2, 2, nbm, nbm), -1, np.int32)
+        ns = np.zeros((2, 2, nbm), np.int32)
+        for i in range(nbm):
+            idx[:, :, i, :i + 1] = np.arange(i + 1)
+            ns[:, :, i] = i + 1
+        out, lse = oracle.prefill_attend(c["q"], c["k"], c["v"], c["lens"], idx, ns, blk)
+        Q, K, V = (torch.from_numpy(widen(c[n])) for n in ("q", "k", "v"))
+        for b, L in enumerate(int(x) for x in c["lens"]):
+            kk = K[b, :, :L].repeat_interleave(c["G"], 0)
+            vv = V[b, :, :L].repeat_interleave(c["G"], 0)
+            ref = torch.nn.functional.scaled_dot_product_attention(Q[b, :, :L], kk, vv, is_causal=True)
+            np.testing.assert_allclose(out[b, :, :L], ref.numpy(), rtol=0, atol=1e-12)
+            z = (Q[b, :, :L] @ kk.transpose(1, 2)) / math.sqrt(Q.shape[-1])
+            z = z.masked_fill(torch.triu(torch.ones(L, L, dtype=torch.bool), 1), float("-inf"))
+            np.testing.assert_allclose(lse[b, :, :L], torch.logsumexp(z, -1).numpy(), rtol=0, atol=1e-12)
+            assert np.all(out[b, :, L:] == 0.0) and np.all(lse[b, :, L:] == -np.inf)
+
+
+def test_prefill_zero_keys_average_kept_causal_values(oracle):
+    c = prefill_case(3, Lmax=64 * 5, lens=(64 * 5, 64 * 3 + 10))
+    c["k"][:] = bits(np.zeros(1, np.float32))[0]
+    idx = np.full((2, 2, 5, 2), -1, np.int32)
+    ns = np.zeros((2, 2, 5), np.int32)
+    for i in range(5):
+        keep = [0, i] if i > 0 else [0]
+        idx[:, :, i, :len(keep)] = keep
+        ns[:, :, i] = len(keep)
+    out, lse = oracle.prefill_attend(c["q"], c["k"], c["v"], c["lens"], idx, ns, 64)
+    V = widen(c["v"])
+    for b, L in enumerate(int(x) for x in c["lens"]):
+        for h in range(4):
+            for t in range(L):
+                i = t // 64
+                toks = [u for j in sorted(set([0, i])) for u in range(j * 64, j * 64 + 64) if u <= t]
+                np.testing.assert_allclose(out[b, h, t], V[b, h // 2, toks].mean(0), rtol=0, atol=1e-12)
+                assert abs(lse[b, h, t] - math.log(len(toks))) < 1e-12
