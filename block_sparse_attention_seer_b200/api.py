@@ -50,6 +50,9 @@ def _load_library():
         "seer_append_kv": [D, P, P, P, P, P, P],
         "seer_block_mass": [D, P, P, P, F32, P, P, P],
         "seer_gate_scores_agg": [D, P, P, P, P, I32, P, P],
+        "seer_prefill_gate_scores": [D, P, P, P, P, P, P],
+        "seer_prefill_select_blocks": [D, P, P, I32, P, P, P],
+        "seer_prefill_attention": [D, P, P, P, P, P, P, I32, F32, P, P, P],
         "seer_select_blocks_threshold": [D, P, P, I32, F32, P, P, P],
         "seer_default_num_splits": [I32, P],
         "seer_decode_wait_failures": [P, I32],
@@ -138,6 +141,29 @@ def seer_sparse_decode(dims, q, k_cache, v_cache, seq_lens, block_idx, num_selec
 def seer_combine(dims, o_part, lse_part, num_splits, out, lse_out, stream=None):
     _check("seer_combine", LIB.seer_combine(ctypes.byref(dims), _ptr(o_part), _ptr(lse_part), int(num_splits),
                                             _ptr(out), _ptr(lse_out), _stream(stream)))
+
+
+def seer_prefill_gate_scores(dims, q, w_q, kpool, seq_lens, scores, stream=None):
+    """Prefill block scores [B, Hkv, NBmax, NBmax] (query block i, key block j <= i)."""
+    _check("seer_prefill_gate_scores", LIB.seer_prefill_gate_scores(ctypes.byref(dims), _ptr(q), _ptr(w_q),
+                                                                    _ptr(kpool), _ptr(seq_lens), _ptr(scores),
+                                                                    _stream(stream)))
+
+
+def seer_prefill_select_blocks(dims, scores, seq_lens, budget_tokens, block_idx, num_selected, stream=None):
+    """Per query block: itself plus the top min(k, i+1)-1 earlier blocks, ascending."""
+    _check("seer_prefill_select_blocks",
+           LIB.seer_prefill_select_blocks(ctypes.byref(dims), _ptr(scores), _ptr(seq_lens), int(budget_tokens),
+                                          _ptr(block_idx), _ptr(num_selected), _stream(stream)))
+
+
+def seer_prefill_attention(dims, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax, out, lse_out=None,
+                           sm_scale=0.0, stream=None):
+    """Causal block-sparse attention of every prompt token over its query block's kept blocks."""
+    _check("seer_prefill_attention",
+           LIB.seer_prefill_attention(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                      _ptr(block_idx), _ptr(num_selected), int(kmax), float(sm_scale), _ptr(out),
+                                      _ptr(lse_out), _stream(stream)))
 
 
 AGG_MEAN, AGG_MAX, AGG_SOFTMAX_MEAN = 0, 1, 2

@@ -180,6 +180,49 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
     return from_cuda(seer::launch_combine(s, o_part, lse_part, num_splits, out, lse_out, stream));
 }
 
+constexpr int kMaxPrefillBlocks = 4096;  // the prefill score matrix is NBmax x NBmax per row
+
+seer_status seer_prefill_gate_scores(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
+                                     const int32_t* seq_lens, float* scores, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !w_q || !kpool || !seq_lens || !scores) return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(w_q, 16) || !aligned(kpool, 16)) return SEER_ERR_INVALID_ARG;
+    if (s.NBmax > kMaxPrefillBlocks) return SEER_ERR_UNSUPPORTED;
+    return from_cuda(seer::launch_prefill_gate(s, q, w_q, kpool, seq_lens, scores, stream));
+}
+
+seer_status seer_prefill_select_blocks(const seer_dims* dims, const float* scores, const int32_t* seq_lens,
+                                       int32_t budget_tokens, int32_t* block_idx, int32_t* num_selected,
+                                       cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!scores || !seq_lens || !block_idx || !num_selected) return SEER_ERR_INVALID_ARG;
+    if (budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
+    if (s.NBmax > kMaxPrefillBlocks) return SEER_ERR_UNSUPPORTED;
+    return from_cuda(
+        seer::launch_prefill_select(s, scores, seq_lens, budget_tokens / s.blk, block_idx, num_selected, stream));
+}
+
+seer_status seer_prefill_attention(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* seq_lens, const int32_t* block_idx, const int32_t* num_selected,
+                                   int32_t kmax, float sm_scale, void* out, float* lse_out, cudaStream_t stream) {
+    Shape s;
+    seer_status st = check_dims(dims, s);
+    if (st != SEER_OK) return st;
+    if (!q || !k_cache || !v_cache || !seq_lens || !block_idx || !num_selected || !out || kmax < 1)
+        return SEER_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4))
+        return SEER_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
+    if (s.NBmax > kMaxPrefillBlocks) return SEER_ERR_UNSUPPORTED;
+    const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
+    return from_cuda(seer::launch_prefill_attention(s, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax,
+                                                    scale, out, lse_out, stream));
+}
+
 seer_status seer_gate_scores_agg(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
                                  const int32_t* seq_lens, int32_t aggregation, float* scores, cudaStream_t stream) {
     Shape s;

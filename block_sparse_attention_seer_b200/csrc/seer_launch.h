@@ -88,6 +88,17 @@ cudaError_t launch_gate_scores_agg(const Shape& s, const void* q, const float* w
 cudaError_t launch_select_threshold(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax, float tau,
                                     int32_t* block_idx, int32_t* num_selected, cudaStream_t stream);
 
+// Block-sparse prefill (prefill.cu): query-block gate scores [B, Hkv, NBmax, NBmax]
+// (j <= i), per-query-block selection [B, Hkv, NBmax, kmax] / [B, Hkv, NBmax], and
+// causal block-sparse attention out bf16 [B, Hq, Lmax, D], lse [B, Hq, Lmax] (nullable).
+cudaError_t launch_prefill_gate(const Shape& s, const void* q, const float* w_q, const float* kpool,
+                                const int32_t* seq_lens, float* scores, cudaStream_t stream);
+cudaError_t launch_prefill_select(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax,
+                                  int32_t* block_idx, int32_t* num_selected, cudaStream_t stream);
+cudaError_t launch_prefill_attention(const Shape& s, const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* seq_lens, const int32_t* block_idx, const int32_t* num_selected,
+                                     int kmax, float sm_scale, void* out, float* lse_out, cudaStream_t stream);
+
 // Block-level ground truth: each query head's dense softmax mass per KV block
 // [B, Hq, NBmax] and lse [B, Hq] (nullable) (block_mass.cu).
 cudaError_t launch_block_mass(const Shape& s, const void* q, const void* k_cache, const int32_t* seq_lens,

@@ -188,6 +188,51 @@ seer_status seer_sparse_decode(const seer_dims* dims, const void* q, const void*
 seer_status seer_combine(const seer_dims* dims, const float* o_part, const float* lse_part,
                          int32_t num_splits, void* out, float* lse_out, cudaStream_t stream);
 
+/* Block-sparse prefill. "SeerAttention: Learning Intrinsic Sparse Attention
+ * in Your LLMs" (abstract): pool Q and K along the sequence, pass them
+ * through the learnable linear layers, multiply into block-level scores and
+ * run a block-sparse attention over the kept blocks. Read for a causal prompt
+ * of L_b tokens (L_b = clamped seq_lens[b]) with query and key blocks of
+ * block_size tokens, the gate and selection readings of the decode path:
+ *
+ * seer_prefill_gate_scores:
+ *   qbar[b, kvh, i] = mean over the group's heads and the valid tokens of
+ *                     query block i of q[b, h, t, :]
+ *   scores[b, kvh, i, j] = (W_q[kvh] qbar) . kpool[b, kvh, j] / sqrt(dg),
+ *                     j <= i < NB_b; other entries are left undefined.
+ *   q        bf16 [B, Hq, Lmax, D]  (16-byte aligned; token t of head h at [b, h, t, :])
+ *   kpool    fp32 [B, Hkv, NBmax, dg]  (seer_kpool_update over the prompt)
+ *   scores   fp32 [B, Hkv, NBmax, NBmax]
+ *
+ * seer_prefill_select_blocks: for each query block i < NB_b, block i itself
+ * plus the top min(k, i + 1) - 1 of blocks 0 .. i-1 (higher score, then lower
+ * index), ascending; k = budget_tokens / block_size. -1 fills the rest; query
+ * blocks i >= NB_b get num_selected 0.
+ *   block_idx     int32 [B, Hkv, NBmax, kmax]
+ *   num_selected  int32 [B, Hkv, NBmax]
+ *
+ * seer_prefill_attention: token t < L_b of query block i = t / block_size,
+ * head h: out = softmax(q_t . K_u * sm_scale) V_u over the tokens u <= t,
+ * u < L_b, of the kept blocks of (b, kvh, i) (entries outside [0, i] are
+ * skipped); lse its natural-log denominator. Rows t >= L_b: out 0, lse -inf.
+ * sm_scale <= 0 means 1/sqrt(D).
+ *   k_cache, v_cache  bf16 [B, Hkv, Lmax, D]
+ *   out               bf16 [B, Hq, Lmax, D]  (output)
+ *   lse_out           fp32 [B, Hq, Lmax]     (output, may be NULL)
+ *
+ * Errors: SEER_ERR_INVALID_ARG for NULL/unaligned pointers, bad budgets or
+ * scales; SEER_ERR_UNSUPPORTED when NBmax > 4096 or outside the supported
+ * sizes.
+ */
+seer_status seer_prefill_gate_scores(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
+                                     const int32_t* seq_lens, float* scores, cudaStream_t stream);
+seer_status seer_prefill_select_blocks(const seer_dims* dims, const float* scores, const int32_t* seq_lens,
+                                       int32_t budget_tokens, int32_t* block_idx, int32_t* num_selected,
+                                       cudaStream_t stream);
+seer_status seer_prefill_attention(const seer_dims* dims, const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* seq_lens, const int32_t* block_idx, const int32_t* num_selected,
+                                   int32_t kmax, float sm_scale, void* out, float* lse_out, cudaStream_t stream);
+
 /* Gate variants. Neither page says how the G query heads of a GQA group share
  * one block score, nor whether a threshold may replace the token budget; the
  * mean gate and top-k above are the plain readings, these are the
