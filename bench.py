@@ -39,6 +39,7 @@ METRIC = "sparse decode attention µs/step and HBM GB/s vs ~8 TB/s at 90% sparsi
 UNIT = "us/step"
 DEFAULT_WORKLOAD = "decode_b16"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sparse_decode_traffic.json")
 # the sources the fused step kernel is compiled from: a recorded traffic figure holds only while they are unchanged
@@ -61,10 +62,34 @@ def parse():
     p.add_argument("--dense-steps", type=int, default=30, help="timed steps of the dense baseline (0: skip)")
     p.add_argument("--mass-steps", type=int, default=30, help="timed calls of the block-level ground truth (0: skip)")
     p.add_argument("--variant-steps", type=int, default=30, help="timed calls of each gate variant (0: skip)")
+    p.add_argument("--prefill-steps", type=int, default=3, help="timed block-sparse prefills (0: skip)")
+    p.add_argument("--prefill-batch", type=int, default=4, help="sequences of the prefill measurement")
     return p.parse_args()
 
 
 # ---------------------------------------------------------------- shared helpers
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def prefill_flops(lens, idx, nsel, blk, D, G):
+    """Useful flops of the causal block-sparse prefill: 4 D per (query token, visible key token) per head."""
+    B, Hkv, nbm, kmax = idx.shape
+    L = np.asarray(lens, np.int64)[:, None, None, None]
+    i = np.arange(nbm, dtype=np.int64)[None, None, :, None]
+    j = idx.astype(np.int64)
+    live = (np.arange(kmax)[None, None, None, :] < nsel[..., None]) & (j >= 0)
+    nq = np.clip(L - i * blk, 0, blk)
+    nk = np.clip(L - j * blk, 0, blk)
+    pairs = np.where(j < i, nq * nk, np.where(j == i, nq * (nq + 1) // 2, 0))
+    return int(4 * D * G * np.where(live, pairs, 0).sum())
+
 
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -487,6 +512,54 @@ def run_ours(args):
         variants["threshold_select_us"] = round(timed(lambda: api.seer_select_blocks_threshold(
             st.dims, vs, inp["seq_lens"], st.budget_tokens, 0.0, thr_idx, thr_ns)), 3)
 
+    # ---- block-sparse prefill over the workload's own caches (the prompt = the cached tokens)
+    prefill = None
+    if args.prefill_steps > 0:
+        pb = min(wl.batch, args.prefill_batch)
+        Hq, Hkv, D, blk = wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+        nbm = wl.nb_max
+        pdims = api.make_dims(pb, Hq, Hkv, D, wl.gate_dim, blk, wl.max_seq_len)
+        gq = torch.Generator(device=dev).manual_seed(args.seed + 7)
+        pq = torch.randn(pb, Hq, wl.max_seq_len, D, generator=gq, device=dev).to(torch.bfloat16)
+        pk, pv = inp["k_cache"][:pb], inp["v_cache"][:pb]
+        plen = inp["seq_lens"][:pb]
+        pkp = st.kpool[:pb]
+        psc = torch.empty(pb, Hkv, nbm, nbm, device=dev)
+        pidx = torch.empty(pb, Hkv, nbm, st.kmax, dtype=torch.int32, device=dev)
+        pns = torch.empty(pb, Hkv, nbm, dtype=torch.int32, device=dev)
+        pout = torch.empty(pb, Hq, wl.max_seq_len, D, dtype=torch.bfloat16, device=dev)
+        plse = torch.empty(pb, Hq, wl.max_seq_len, device=dev)
+        calls = {
+            "gate": lambda: api.seer_prefill_gate_scores(pdims, pq, inp["w_q"], pkp, plen, psc),
+            "select": lambda: api.seer_prefill_select_blocks(pdims, psc, plen, wl.budget_tokens, pidx, pns),
+            "attention": lambda: api.seer_prefill_attention(pdims, pq, pk, pv, plen, pidx, pns, st.kmax, pout, plse),
+        }
+        times = {}
+        for name, fn in calls.items():
+            p_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.prefill_steps)]
+            for kk in range(args.prefill_steps + 1):
+                prepare()
+                evs = p_ev[kk - 1] if kk >= 1 else None
+                if evs:
+                    evs[0].record(stream)
+                fn()
+                if evs:
+                    evs[1].record(stream)
+            torch.cuda.synchronize()
+            t_us = float(np.mean([e[0].elapsed_time(e[1]) for e in p_ev])) * 1e3
+            times[name] = max_over_ranks([t_us], dev)[0] if world > 1 else t_us
+        flops = prefill_flops(lens[:pb], pidx.cpu().numpy(), pns.cpu().numpy(), blk, D, wl.group)
+        tpeak, tkind = measured_tensor_peak()
+        tflops = flops / (times["attention"] * 1e-6) / 1e12
+        prefill = {"batch": pb, "prompt_tokens": [int(x) for x in lens[:pb]],
+                   "gate_us": round(times["gate"], 1), "select_us": round(times["select"], 1),
+                   "attention_us": round(times["attention"], 1), "attention_flops": flops,
+                   "attention_tflops": round(tflops, 1), "bound": "tensor", "peak_tflops": tpeak,
+                   "peak_kind": tkind, "frac": round(tflops / tpeak, 4),
+                   "flops_counted": "4 D per (query token, causally visible key token of a kept block) per head"}
+        del pq, psc, pidx, pns, pout, plse
+        torch.cuda.empty_cache()
+
     # ---- end to end through the public API: host inputs in, host output out, every step.
     # The step's inputs (q and the new token's K/V rows) travel as one packed pinned buffer;
     # seer_append_kv places the token in the caches, the fused step runs, out comes back.
@@ -555,6 +628,7 @@ def run_ours(args):
             "dense_baseline": dense,
             "block_mass": block_mass,
             "gate_variants": variants,
+            "prefill": prefill,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
