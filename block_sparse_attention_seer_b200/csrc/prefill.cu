@@ -16,7 +16,8 @@
 //           the tokens u <= t (u < L_b) of the kept blocks of (b, kvh, i)
 //
 // prefill_gate_kernel / prefill_select_kernel: one CTA per (row, query block).
-// prefill_attn_kernel: one CTA per (b, query head, query block), 16 query
+// prefill_attn_kernel: one CTA per (b, query head, query block), the heads of
+// a group launched side by side so they share K/V tiles through L2, 16 query
 // rows per warp, FlashAttention-style online softmax on mma.sync (S = Q K^T
 // and O += P V, the S accumulators re-packed as the A operand of P V), K/V
 // tiles double-buffered in shared memory by cp.async; rows past L_b are
@@ -155,10 +156,14 @@ __global__ void __launch_bounds__(PrefillCfg<D, BLK>::kThreads, 1)
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tig = lane & 3;
-    const int i = blockIdx.x, bh = blockIdx.y;
-    const int b = bh / Hq, hq = bh - b * Hq;
-    const int kvh = hq / (Hq / Hkv);
-    const int row = b * Hkv + kvh;
+    // blockIdx.x = query block * G + head of the group: the G heads reading the
+    // same K/V tiles (and the next query blocks, which keep mostly the same
+    // blocks) launch next to each other, so the tiles are shared through L2
+    const int G = Hq / Hkv;
+    const int i = blockIdx.x / G, row = blockIdx.y;
+    const int b = row / Hkv, kvh = row - b * Hkv;
+    const int hq = kvh * G + (blockIdx.x - i * G);
+    const int bh = b * Hq + hq;
     const int L = clamp_len(seq_lens[b], Lmax);
     const int t0 = i * BLK;
     const int r0 = t0 + warp * 16 + g, r1 = r0 + 8;  // this lane's two query rows
@@ -365,7 +370,7 @@ cudaError_t attn_impl(const Shape& s, const void* q, const void* k_cache, const 
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    prefill_attn_kernel<D, BLK><<<dim3(s.NBmax, s.B * s.Hq), C::kThreads, C::kSmem, stream>>>(
+    prefill_attn_kernel<D, BLK><<<dim3(s.NBmax * s.G, s.B * s.Hkv), C::kThreads, C::kSmem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
         static_cast<const __nv_bfloat16*>(v_cache), seq_lens, block_idx, num_selected, s.Hq, s.Hkv, s.Lmax, s.NBmax,
         kmax, sm_scale * kLog2e, static_cast<__nv_bfloat16*>(out), lse_out);

@@ -189,7 +189,7 @@ seer_status seer_prefill_gate_scores(const seer_dims* dims, const void* q, const
     if (st != SEER_OK) return st;
     if (!q || !w_q || !kpool || !seq_lens || !scores) return SEER_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(w_q, 16) || !aligned(kpool, 16)) return SEER_ERR_INVALID_ARG;
-    if (s.NBmax > kMaxPrefillBlocks) return SEER_ERR_UNSUPPORTED;
+    if (s.NBmax > kMaxPrefillBlocks || s.B * s.Hkv > 65535) return SEER_ERR_UNSUPPORTED;  // grid y = rows
     return from_cuda(seer::launch_prefill_gate(s, q, w_q, kpool, seq_lens, scores, stream));
 }
 
@@ -201,7 +201,7 @@ seer_status seer_prefill_select_blocks(const seer_dims* dims, const float* score
     if (st != SEER_OK) return st;
     if (!scores || !seq_lens || !block_idx || !num_selected) return SEER_ERR_INVALID_ARG;
     if (budget_tokens < s.blk || budget_tokens % s.blk != 0) return SEER_ERR_INVALID_ARG;
-    if (s.NBmax > kMaxPrefillBlocks) return SEER_ERR_UNSUPPORTED;
+    if (s.NBmax > kMaxPrefillBlocks || s.B * s.Hkv > 65535) return SEER_ERR_UNSUPPORTED;  // grid y = rows
     return from_cuda(
         seer::launch_prefill_select(s, scores, seq_lens, budget_tokens / s.blk, block_idx, num_selected, stream));
 }
@@ -217,7 +217,7 @@ seer_status seer_prefill_attention(const seer_dims* dims, const void* q, const v
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4))
         return SEER_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
-    if (s.NBmax > kMaxPrefillBlocks) return SEER_ERR_UNSUPPORTED;
+    if (s.NBmax > kMaxPrefillBlocks || s.B * s.Hkv > 65535) return SEER_ERR_UNSUPPORTED;  // grid y = rows
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
     return from_cuda(seer::launch_prefill_attention(s, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax,
                                                     scale, out, lse_out, stream));

@@ -221,7 +221,7 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
  *   lse_out           fp32 [B, Hq, Lmax]     (output, may be NULL)
  *
  * Errors: SEER_ERR_INVALID_ARG for NULL/unaligned pointers, bad budgets or
- * scales; SEER_ERR_UNSUPPORTED when NBmax > 4096 or outside the supported
+ * scales; SEER_ERR_UNSUPPORTED when NBmax > 4096, batch x num_kv_heads > 65535 or outside the supported
  * sizes.
  */
 seer_status seer_prefill_gate_scores(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
