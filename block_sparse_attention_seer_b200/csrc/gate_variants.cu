@@ -16,14 +16,19 @@
 //   threshold:     block NB_b - 1, plus the candidates with s >= tau, at most
 //                  k_b - 1 of them (the highest, equal scores to the lower index)
 //
-// One CTA per (b, kv head) row for both. Scores: the group's projected
-// queries in shared memory, then lane quads score pooled-K rows (the order of
-// gate_core.cuh's quad_row_dot); the softmax mean takes three passes over the
-// row (max, sum, scores), the later ones L2-resident.
+// Scores: a cluster of CTAs per (b, kv head) row shares the group's projected
+// queries through distributed shared memory and splits the row; lane quads
+// score pooled-K rows (the order of gate_core.cuh's quad_row_dot); the
+// softmax mean takes three passes over its chunk (max, sum, scores), the
+// later ones L2-resident. Threshold selection: one CTA per row.
 #include <cuda_bf16.h>
+
+#include <cooperative_groups.h>
 
 #include "gate_core.cuh"
 #include "seer_launch.h"
+
+namespace cg = cooperative_groups;
 
 namespace seer {
 namespace {
@@ -31,30 +36,41 @@ namespace {
 constexpr int kAggThreads = 256;
 constexpr int kAggWarps = kAggThreads / 32;
 constexpr int kMaxG = 8;
+constexpr int kMaxCluster = 8;
 
+// A thread-block cluster of C CTAs per row: each CTA projects dg / C
+// components of every head's query and the cluster exchanges them through
+// distributed shared memory; each CTA then scores its own contiguous chunk of
+// the row. The softmax mean combines each head's chunk maxima, then chunk sums,
+// across the cluster the same way.
 template <int D, int DG>
 __global__ void __launch_bounds__(kAggThreads)
     gate_scores_agg_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w_q,
                            const float* __restrict__ kpool, const int32_t* __restrict__ seq_lens, int Hq, int Hkv,
                            int Lmax, int blk, int NBmax, int agg, float* __restrict__ scores) {
     __shared__ __align__(16) float qh[kMaxG][D];
+    __shared__ float qg_part[kMaxG][DG];          // components this CTA projects
     __shared__ __align__(16) float qg[kMaxG][DG];
     __shared__ float red[kAggWarps][kMaxG];
+    __shared__ float part[kMaxG];                 // this CTA's per-head max, then sum (read by the cluster)
     __shared__ float hmax[kMaxG], hsum[kMaxG];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int csize = (int)cluster.num_blocks();
+    const int crank = (int)cluster.block_rank();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = lane >> 2, qlane = lane & 3;
-    const int row = blockIdx.x;
+    const int row = blockIdx.y;
     const int b = row / Hkv, kvh = row - b * Hkv;
     const int G = Hq / Hkv;
     const int NB = (clamp_len(seq_lens[b], Lmax) + blk - 1) / blk;
     const float inv_sqrt_dg = 1.0f / sqrtf((float)DG);
 
-    for (int i = tid; i < G * D; i += kAggThreads)
-        qh[i / D][i % D] = __bfloat162float(q[((size_t)b * Hq + (size_t)kvh * G) * D + i]);
+    for (int x = tid; x < G * D; x += kAggThreads)
+        qh[x / D][x % D] = __bfloat162float(q[((size_t)b * Hq + (size_t)kvh * G) * D + x]);
     __syncthreads();
-    // projections: warp w takes outputs e = w, w + 8, ...; one W_q row serves every head
     const float* W = w_q + (size_t)kvh * DG * D;
-    for (int e = warp; e < DG; e += kAggWarps) {
+    const int per_e = DG / csize;
+    for (int e = crank * per_e + warp; e < (crank + 1) * per_e; e += kAggWarps) {
         float wv[D / 32];
 #pragma unroll
         for (int u = 0; u < D / 32; ++u) wv[u] = W[(size_t)e * D + lane + 32 * u];
@@ -63,62 +79,75 @@ __global__ void __launch_bounds__(kAggThreads)
 #pragma unroll
             for (int u = 0; u < D / 32; ++u) acc = fmaf(wv[u], qh[h][lane + 32 * u], acc);
             acc = warp_sum(acc);
-            if (lane == 0) qg[h][e] = acc;
+            if (lane == 0) qg_part[h][e] = acc;
         }
     }
-    __syncthreads();
+    cluster.sync();
+    for (int x = tid; x < G * DG; x += kAggThreads) {
+        const int h = x / DG, e = x - h * DG;
+        qg[h][e] = *cluster.map_shared_rank(&qg_part[h][e], e / per_e);
+    }
+    cluster.sync();  // remote reads done before qg_part could be left behind
 
+    const int per = (NB + csize - 1) / csize;
+    const int j0 = crank * per, j1 = min(NB, j0 + per);
     const float* kp = kpool + (size_t)row * NBmax * DG;
     float* out = scores + (size_t)row * NBmax;
-    // score of head h at block j (every lane of the quad gets it)
     auto head_score = [&](int j, int h) { return quad_row_dot<DG>(kp + (size_t)j * DG, j, qg[h], qlane) * inv_sqrt_dg; };
     if (agg == 2) {
-        // pass 1: each head's max over the row; pass 2: its sum of exponentials
+        // pass 0: each head's max over the row; pass 1: its sum of exponentials
         for (int pass = 0; pass < 2; ++pass) {
             float acc[kMaxG];
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) acc[h] = pass == 0 ? -INFINITY : 0.f;
-            for (int j0 = warp * 8; j0 < NB; j0 += kAggWarps * 8) {
-                const int j = min(j0 + quad, NB - 1);
-                const bool live = j0 + quad < NB;
+            for (int jb = j0 + warp * 8; jb < j1; jb += kAggWarps * 8) {
+                const int j = min(jb + quad, j1 - 1);
+                const bool live = jb + quad < j1;
 #pragma unroll
                 for (int h = 0; h < kMaxG; ++h) {
                     if (h >= G) break;
-                    const float s = head_score(j, h);
-                    if (live) acc[h] = pass == 0 ? fmaxf(acc[h], s) : acc[h] + expf(s - hmax[h]);
+                    const float sc = head_score(j, h);
+                    if (live) acc[h] = pass == 0 ? fmaxf(acc[h], sc) : acc[h] + expf(sc - hmax[h]);
                 }
             }
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) {
                 if (h >= G) break;
-                float v = acc[h];
-                if (pass == 0) v = warp_max(v);
-                else v = warp_sum(qlane == 0 ? v : 0.f);  // the quad's 4 lanes hold the same terms
+                const float v = pass == 0 ? warp_max(acc[h]) : warp_sum(qlane == 0 ? acc[h] : 0.f);
                 if (lane == 0) red[warp][h] = v;
             }
             __syncthreads();
             if (tid < G) {
                 float v = pass == 0 ? -INFINITY : 0.f;
                 for (int w = 0; w < kAggWarps; ++w) v = pass == 0 ? fmaxf(v, red[w][tid]) : v + red[w][tid];
+                part[tid] = v;
+            }
+            cluster.sync();
+            if (tid < G) {
+                float v = pass == 0 ? -INFINITY : 0.f;
+                for (int c = 0; c < csize; ++c) {
+                    const float pc = *cluster.map_shared_rank(&part[tid], c);
+                    v = pass == 0 ? fmaxf(v, pc) : v + pc;
+                }
                 if (pass == 0) hmax[tid] = v;
                 else hsum[tid] = v;
             }
-            __syncthreads();
+            cluster.sync();  // remote reads of `part` done before it is rewritten or the CTA exits
         }
     }
-    for (int j0 = warp * 8; j0 < NB; j0 += kAggWarps * 8) {
-        const int j = min(j0 + quad, NB - 1);
+    for (int jb = j0 + warp * 8; jb < j1; jb += kAggWarps * 8) {
+        const int j = min(jb + quad, j1 - 1);
         float a = agg == 1 ? -INFINITY : 0.f;
 #pragma unroll
         for (int h = 0; h < kMaxG; ++h) {
             if (h >= G) break;
-            const float s = head_score(j, h);
-            if (agg == 1) a = fmaxf(a, s);
-            else if (agg == 2) a += expf(s - hmax[h]) / hsum[h];
-            else a += s;
+            const float sc = head_score(j, h);
+            if (agg == 1) a = fmaxf(a, sc);
+            else if (agg == 2) a += expf(sc - hmax[h]) / hsum[h];
+            else a += sc;
         }
         if (agg != 1) a /= (float)G;
-        if (qlane == 0 && j0 + quad < NB) out[j] = a;
+        if (qlane == 0 && jb + quad < j1) out[j] = a;
     }
 }
 
@@ -162,23 +191,37 @@ __global__ void __launch_bounds__(kSelThreads)
     if (NB > 0) select_row<kSelThreads>(keys, NB, keep, out, sm);
 }
 
+template <int D, int DG>
+cudaError_t agg_impl(const Shape& s, const void* q, const float* w_q, const float* kpool, const int32_t* seq_lens,
+                     int agg, float* scores, int csize, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize, s.B * s.Hkv, 1);
+    cfg.blockDim = dim3(kAggThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gate_scores_agg_kernel<D, DG>, static_cast<const __nv_bfloat16*>(q),
+                                             w_q, kpool, seq_lens, s.Hq, s.Hkv, s.Lmax, s.blk, s.NBmax, agg, scores);
+    if (e != cudaSuccess) (void)cudaGetLastError();  // a rejected launch must not leak into the next call
+    return e;
+}
+
 }  // namespace
 
 cudaError_t launch_gate_scores_agg(const Shape& s, const void* q, const float* w_q, const float* kpool,
-                                   const int32_t* seq_lens, int agg, float* scores, cudaStream_t stream) {
-    const auto* qb = static_cast<const __nv_bfloat16*>(q);
-    const dim3 grid(s.B * s.Hkv);
-#define SEER_AGG_CASE(DV, DGV)                                                                                  \
-    if (s.D == DV && s.dg == DGV) {                                                                             \
-        gate_scores_agg_kernel<DV, DGV><<<grid, kAggThreads, 0, stream>>>(qb, w_q, kpool, seq_lens, s.Hq, s.Hkv, \
-                                                                          s.Lmax, s.blk, s.NBmax, agg, scores); \
-        return cudaGetLastError();                                                                              \
-    }
-    SEER_AGG_CASE(128, 128)
-    SEER_AGG_CASE(128, 64)
-    SEER_AGG_CASE(64, 128)
-    SEER_AGG_CASE(64, 64)
-#undef SEER_AGG_CASE
+                                   const int32_t* seq_lens, int agg, float* scores, int num_sms, cudaStream_t stream) {
+    const int rows = s.B * s.Hkv;
+    int csize = 1;  // enough CTAs for every SM, at least 32 blocks per CTA
+    while (csize < kMaxCluster && rows * csize < 2 * num_sms && s.NBmax / (2 * csize) >= 32) csize *= 2;
+    if (s.D == 128 && s.dg == 128) return agg_impl<128, 128>(s, q, w_q, kpool, seq_lens, agg, scores, csize, stream);
+    if (s.D == 128 && s.dg == 64) return agg_impl<128, 64>(s, q, w_q, kpool, seq_lens, agg, scores, csize, stream);
+    if (s.D == 64 && s.dg == 128) return agg_impl<64, 128>(s, q, w_q, kpool, seq_lens, agg, scores, csize, stream);
+    if (s.D == 64 && s.dg == 64) return agg_impl<64, 64>(s, q, w_q, kpool, seq_lens, agg, scores, csize, stream);
     return cudaErrorInvalidValue;
 }
 

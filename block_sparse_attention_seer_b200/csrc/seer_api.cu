@@ -231,7 +231,8 @@ seer_status seer_gate_scores_agg(const seer_dims* dims, const void* q, const flo
     if (!q || !w_q || !kpool || !seq_lens || !scores) return SEER_ERR_INVALID_ARG;
     if (aggregation < SEER_AGG_MEAN || aggregation > SEER_AGG_SOFTMAX_MEAN) return SEER_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(w_q, 16) || !aligned(kpool, 16)) return SEER_ERR_INVALID_ARG;
-    return from_cuda(seer::launch_gate_scores_agg(s, q, w_q, kpool, seq_lens, aggregation, scores, stream));
+    return from_cuda(
+        seer::launch_gate_scores_agg(s, q, w_q, kpool, seq_lens, aggregation, scores, device_sm_count(), stream));
 }
 
 seer_status seer_select_blocks_threshold(const seer_dims* dims, const float* scores, const int32_t* seq_lens,

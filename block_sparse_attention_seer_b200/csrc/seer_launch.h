@@ -84,7 +84,7 @@ cudaError_t run_wait_selftest(unsigned long long limit_ns, int* timed_out);
 // (0 mean, 1 max, 2 mean of each head's softmax over its row's blocks), and
 // threshold selection (at most kmax - 1 candidates scoring >= tau, plus the last block).
 cudaError_t launch_gate_scores_agg(const Shape& s, const void* q, const float* w_q, const float* kpool,
-                                   const int32_t* seq_lens, int agg, float* scores, cudaStream_t stream);
+                                   const int32_t* seq_lens, int agg, float* scores, int num_sms, cudaStream_t stream);
 cudaError_t launch_select_threshold(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax, float tau,
                                     int32_t* block_idx, int32_t* num_selected, cudaStream_t stream);
 
