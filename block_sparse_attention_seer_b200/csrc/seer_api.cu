@@ -85,17 +85,22 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D view [B*Hkv*Lmax rows, D cols] of a bf16 cache; box = 64 cols (128 B) x blk rows, 128-byte swizzle.
-bool encode_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+// 2-D view [rows, D cols] of a bf16 tensor; box = 64 cols (128 B) x box_rows rows, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* m, const void* base, int D, long long rows, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)s.D, (cuuint64_t)s.B * s.Hkv * s.Lmax};
-    const cuuint64_t strides[1] = {(cuuint64_t)s.D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)s.blk};
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A bf16 cache [B*Hkv*Lmax rows, D cols] with a blk-row box.
+bool encode_cache_map(CUtensorMap* m, const void* base, const Shape& s) {
+    return encode_rows_map(m, base, s.D, (long long)s.B * s.Hkv * s.Lmax, s.blk);
 }
 
 }  // namespace
@@ -214,13 +219,19 @@ seer_status seer_prefill_attention(const seer_dims* dims, const void* q, const v
     if (st != SEER_OK) return st;
     if (!q || !k_cache || !v_cache || !seq_lens || !block_idx || !num_selected || !out || kmax < 1)
         return SEER_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 4))
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
         return SEER_ERR_INVALID_ARG;
     if (!(sm_scale == sm_scale) || std::isinf(sm_scale)) return SEER_ERR_INVALID_ARG;
     if (s.NBmax > kMaxPrefillBlocks || s.B * s.Hkv > 65535) return SEER_ERR_UNSUPPORTED;  // grid y = rows
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / std::sqrt((float)s.D);
-    return from_cuda(seer::launch_prefill_attention(s, q, k_cache, v_cache, seq_lens, block_idx, num_selected, kmax,
-                                                    scale, out, lse_out, stream));
+    if ((long long)s.B * s.Hq * s.Lmax >= (1LL << 31)) return SEER_ERR_UNSUPPORTED;  // 32-bit TMA row coordinate
+    CUtensorMap tmq, tmk, tmv;
+    if (!encode_rows_map(&tmq, q, s.D, (long long)s.B * s.Hq * s.Lmax, s.blk) ||
+        !encode_rows_map(&tmk, k_cache, s.D, (long long)s.B * s.Hkv * s.Lmax, 64) ||
+        !encode_rows_map(&tmv, v_cache, s.D, (long long)s.B * s.Hkv * s.Lmax, 64))
+        return SEER_ERR_CUDA;
+    return from_cuda(seer::launch_prefill_attention(s, tmq, tmk, tmv, seq_lens, block_idx, num_selected, kmax, scale,
+                                                    out, lse_out, stream));
 }
 
 seer_status seer_gate_scores_agg(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,

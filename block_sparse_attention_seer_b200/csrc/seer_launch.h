@@ -95,9 +95,13 @@ cudaError_t launch_prefill_gate(const Shape& s, const void* q, const float* w_q,
                                 const int32_t* seq_lens, float* scores, cudaStream_t stream);
 cudaError_t launch_prefill_select(const Shape& s, const float* scores, const int32_t* seq_lens, int kmax,
                                   int32_t* block_idx, int32_t* num_selected, cudaStream_t stream);
-cudaError_t launch_prefill_attention(const Shape& s, const void* q, const void* k_cache, const void* v_cache,
-                                     const int32_t* seq_lens, const int32_t* block_idx, const int32_t* num_selected,
-                                     int kmax, float sm_scale, void* out, float* lse_out, cudaStream_t stream);
+// Attention (prefill_attn.cu, tcgen05): tmQ views q as [B*Hq*Lmax, D] with a
+// 64-column x blk-row box, tmK / tmV view the caches as [B*Hkv*Lmax, D] with a
+// 64 x 64 box; all 128-byte swizzled.
+cudaError_t launch_prefill_attention(const Shape& s, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                     const CUtensorMap& tmV, const int32_t* seq_lens, const int32_t* block_idx,
+                                     const int32_t* num_selected, int kmax, float sm_scale, void* out, float* lse_out,
+                                     cudaStream_t stream);
 
 // Block-level ground truth: each query head's dense softmax mass per KV block
 // [B, Hq, NBmax] and lse [B, Hq] (nullable) (block_mass.cu).

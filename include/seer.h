@@ -215,14 +215,17 @@ seer_status seer_combine(const seer_dims* dims, const float* o_part, const float
  * head h: out = softmax(q_t . K_u * sm_scale) V_u over the tokens u <= t,
  * u < L_b, of the kept blocks of (b, kvh, i) (entries outside [0, i] are
  * skipped); lse its natural-log denominator. Rows t >= L_b: out 0, lse -inf.
- * sm_scale <= 0 means 1/sqrt(D).
+ * sm_scale <= 0 means 1/sqrt(D). Runs on the tcgen05 tensor cores (bf16
+ * products, fp32 accumulation; P rounded to bf16 for P V). A bounded wait that
+ * gives up leaves NaN in the rows of the CTA concerned.
+ *   q, k_cache, v_cache  16-byte aligned
  *   k_cache, v_cache  bf16 [B, Hkv, Lmax, D]
- *   out               bf16 [B, Hq, Lmax, D]  (output)
+ *   out               bf16 [B, Hq, Lmax, D]  (output, 16-byte aligned)
  *   lse_out           fp32 [B, Hq, Lmax]     (output, may be NULL)
  *
  * Errors: SEER_ERR_INVALID_ARG for NULL/unaligned pointers, bad budgets or
- * scales; SEER_ERR_UNSUPPORTED when NBmax > 4096, batch x num_kv_heads > 65535 or outside the supported
- * sizes.
+ * scales; SEER_ERR_UNSUPPORTED when NBmax > 4096, batch x num_kv_heads > 65535,
+ * batch x num_q_heads x max_seq_len >= 2^31 or outside the supported sizes.
  */
 seer_status seer_prefill_gate_scores(const seer_dims* dims, const void* q, const float* w_q, const float* kpool,
                                      const int32_t* seq_lens, float* scores, cudaStream_t stream);

@@ -1,4 +1,5 @@
-"""Block-sparse prefill on the GPU against the oracle.
+"""Block-sparse prefill on the GPU against the oracle (attention on the tcgen05
+tensor cores: two M = 128 query tiles per CTA, 64-token key sub-tiles).
 
 * gate scores (query block i, key block j <= i < NB_b): |err| <= 2e-6 (an
   fp32 mean over the group's and the block's queries, one projection, a dot
@@ -104,6 +105,10 @@ def check(c, budget, dense=False):
     (1, 4, 1, 64, 64, 64, 448, [448], 64),
     (3, 4, 2, 64, 128, 128, 512, [512, 0, 129], 128),
     (1, 10, 2, 128, 128, 64, 1024, [1000], 256),
+    (2, 2, 2, 128, 128, 64, 512, [400, 512], 128),      # one head per group: half an M tile
+    (1, 8, 1, 128, 64, 64, 640, [640], 192),            # eight heads: two CTAs per query block
+    (2, 4, 2, 128, 128, 64, 500, [500, 77], 128),       # Lmax not a multiple of the block
+    (1, 4, 1, 64, 64, 128, 640, [577], 256),            # D 64, blk 128, a ragged last block
 ])
 def test_prefill_matches_oracle(shape):
     B, Hq, Hkv, D, dg, blk, Lmax, lens, budget = shape
