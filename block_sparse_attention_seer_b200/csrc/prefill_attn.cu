@@ -48,6 +48,7 @@ constexpr int kMaxAttnStages = 8;
 constexpr float kLog2eA = 1.44269504088896340736f;
 constexpr float kLn2A = 0.69314718055994530942f;
 constexpr float kRescaleLog2 = 8.0f;  // move the reference maximum only past a 2^8 growth
+constexpr int kListCap = 384;         // kept lists up to this length are staged in shared memory
 
 template <int D>
 struct AttnCfg {
@@ -57,7 +58,7 @@ struct AttnCfg {
     static constexpr int kKV = kBoxes * kSub * 128;     // K (or V) of one sub-tile
     static constexpr int kStage = 2 * kKV;
     static constexpr int kFixed = 2 * kQTile + 2 * kPTile;
-    static constexpr int kBarBytes = 256;
+    static constexpr int kBarBytes = 256 + kListCap * 4;
     static constexpr int kStages0 = (kAttnSmemLimit - 1024 - kBarBytes - kFixed) / kStage;
     static constexpr int kStages = kStages0 > kMaxAttnStages ? kMaxAttnStages : kStages0;
     static constexpr int kSmem = 1024 + kFixed + kStages * kStage + kBarBytes;
@@ -100,6 +101,13 @@ struct AttnBars {
     uint32_t q_full, kv_full, kv_empty, s_ready, s_free, p_ready, pv_done, drain;
     // kv_full / kv_empty: + 8 * stage; s_ready / s_free: + 8 * (2 * tile + buffer); p_ready / pv_done: + 8 * tile
 };
+
+// 2^x on the special-function unit (flush-to-zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ bool abort_set(const int* flag) { return *(volatile const int*)flag != 0; }
 
@@ -161,6 +169,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t bar_end = bars.drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + (bar_end - sBar));
     int* abort_flag = reinterpret_cast<int*>(gBar + (bar_end - sBar) + 4);
+    int32_t* list_s = reinterpret_cast<int32_t*>(gBar + 256);
 
     if (tid == 0) {
         mbar_init(bars.q_full, 1);
@@ -184,13 +193,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc::tmem_alloc(smem_addr(tmem_slot), kTmemCols);
         tc::tmem_relinquish();
     }
+    const int32_t* list_g = block_idx + ((size_t)row * NBmax + i) * kmax;
+    const int nsel = min(max(num_selected[(size_t)row * NBmax + i], 0), kmax);
+    for (int x = tid; x < nsel && nsel <= kListCap; x += kAttnThreads) list_s[x] = list_g[x];
+    const int32_t* list = nsel <= kListCap ? list_s : list_g;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-    const int32_t* list = block_idx + ((size_t)row * NBmax + i) * kmax;
-    const int nsel = min(max(num_selected[(size_t)row * NBmax + i], 0), kmax);
     SubIter it0;
     it0.list = list;
     it0.nsel = nsel;
@@ -251,24 +262,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             constexpr uint32_t kIdS = tc::idesc_bf16_f32(128, kSub, false);
             constexpr uint32_t kIdO = tc::idesc_bf16_f32(128, D, true);
             bool ok = mbar_wait(bars.q_full, 0u);
+            const uint64_t dq0 = tc::smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t dq1 = tc::smem_desc_sw128(sQ + C::kQTile, 16, 1024);
+            const uint64_t dp0 = tc::smem_desc_sw128(sP, 16, 1024);
+            const uint64_t dp1 = tc::smem_desc_sw128(sP + C::kPTile, 16, 1024);
             // S_t(n) = Q_t K(n)^T into buffer n % 2 of tile t
             auto issue_s = [&](int n) -> bool {
                 const int st = n % C::kStages;
                 if (!mbar_wait(bars.kv_full + 8 * st, (uint32_t)((n / C::kStages) & 1))) return false;
-                const uint32_t sk = sKV + st * C::kStage;
+                const uint64_t dk = tc::smem_desc_sw128(sKV + st * C::kStage, 16, 1024);
                 for (int t = 0; t < n_tiles; ++t) {
                     const int buf = n & 1;
                     if (n >= 2 && !mbar_wait(bars.s_free + 8 * (2 * t + buf), (uint32_t)(((n - 2) >> 1) & 1)))
                         return false;
                     tc::fence_after_sync();
                     const uint32_t d_tmem = tmem + (uint32_t)(t * (kTmemCols / 2) + D + buf * kSub);
+                    const uint64_t dq = t == 0 ? dq0 : dq1;
+                    // k-th 16-column step: box k / 4, 32 bytes * (k % 4) into the swizzled row
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t a = sQ + t * C::kQTile + (k >> 2) * (128 * 128) + (k & 3) * 32;
-                        const uint32_t bk = sk + (k >> 2) * (kSub * 128) + (k & 3) * 32;
-                        tc::mma_bf16_ss(d_tmem, tc::smem_desc_sw128(a, 16, 1024), tc::smem_desc_sw128(bk, 16, 1024),
-                                        kIdS, k > 0);
-                    }
+                    for (int k = 0; k < D / 16; ++k)
+                        tc::mma_bf16_ss(d_tmem, dq + (uint64_t)((k >> 2) * (128 * 128 / 16) + (k & 3) * 2),
+                                        dk + (uint64_t)((k >> 2) * (kSub * 128 / 16) + (k & 3) * 2), kIdS, k > 0);
                     tc::commit(bars.s_ready + 8 * (2 * t + buf));
                 }
                 return true;
@@ -283,7 +297,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     ok = issue_s(n + 1);
                     if (!ok) break;
                 }
-                const uint32_t sv = sKV + (n % C::kStages) * C::kStage + C::kKV;
+                const uint64_t dv = tc::smem_desc_sw128(sKV + (n % C::kStages) * C::kStage + C::kKV, kSub * 128, 1024);
                 for (int t = 0; t < n_tiles; ++t) {
                     if (!mbar_wait(bars.p_ready + 8 * t, (uint32_t)(n & 1))) {
                         ok = false;
@@ -291,13 +305,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                     tc::fence_after_sync();
                     const uint32_t o_tmem = tmem + (uint32_t)(t * (kTmemCols / 2));
+                    const uint64_t dp = t == 0 ? dp0 : dp1;
+                    // k-th 16-token step: 32 bytes into each P row, 16 V rows further
 #pragma unroll
-                    for (int k = 0; k < kSub / 16; ++k) {
-                        const uint32_t a = sP + t * C::kPTile + k * 32;
-                        const uint32_t bv = sv + k * (16 * 128);
-                        tc::mma_bf16_ss(o_tmem, tc::smem_desc_sw128(a, 16, 1024),
-                                        tc::smem_desc_sw128(bv, kSub * 128, 1024), kIdO, n > 0 || k > 0);
-                    }
+                    for (int k = 0; k < kSub / 16; ++k)
+                        tc::mma_bf16_ss(o_tmem, dp + (uint64_t)(k * 2), dv + (uint64_t)(k * (16 * 128 / 16)), kIdO,
+                                        n > 0 || k > 0);
                     tc::commit(bars.pv_done + 8 * t);
                 }
                 if (!ok) break;
@@ -346,33 +359,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.s_free + 8 * (2 * t + buf));
-            // mask and scale (log2 domain)
+            // mask (only the diagonal and the sequence end), then the row maximum of the raw scores
             const int lim = lim_tok - it.tok0();   // columns 0 .. lim are visible
-            float mx = -INFINITY;
+            if (!__all_sync(0xffffffffu, lim >= kSub - 1)) {
 #pragma unroll
-            for (int c = 0; c < kSub; ++c) {
-                float v = __uint_as_float(s[c >> 5][c & 31]) * scale_log2;
-                v = c <= lim ? v : -INFINITY;
-                s[c >> 5][c & 31] = __float_as_uint(v);
-                mx = fmaxf(mx, v);
+                for (int c = 0; c < kSub; ++c)
+                    if (c > lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < kSub; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(s[c >> 5][c & 31]));
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * scale_log2;  // scale > 0
             float alpha = 1.f;
             if (mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx > -INFINITY)) {
-                alpha = m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx);
+                alpha = m_ref == -INFINITY ? 0.f : ex2(m_ref - mx);
                 m_ref = mx;
                 l *= alpha;
             }
-            const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+            const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
             uint32_t pk[kSub / 2];
-            float sum = 0.f;
+            float sum2[2] = {0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < kSub; c += 2) {
-                const float p0 = exp2f(__uint_as_float(s[c >> 5][c & 31]) - m_use);
-                const float p1 = exp2f(__uint_as_float(s[(c + 1) >> 5][(c + 1) & 31]) - m_use);
-                sum += p0 + p1;
+                const float p0 = ex2(fmaf(__uint_as_float(s[c >> 5][c & 31]), scale_log2, neg_m));
+                const float p1 = ex2(fmaf(__uint_as_float(s[(c + 1) >> 5][(c + 1) & 31]), scale_log2, neg_m));
+                sum2[(c >> 1) & 1] += p0 + p1;
                 pk[c / 2] = pack_bf16x2(p0, p1);
             }
-            l += sum;
+            l += sum2[0] + sum2[1];
             // P and O are free once the previous P V has completed
             if (n > 0) {
                 w = mbar_wait(bars.pv_done + 8 * t, (uint32_t)((n - 1) & 1));
