@@ -10,20 +10,25 @@
 // Design (one CTA per (b, kvh, query block, group of heads)):
 //  * the CTA's query rows -- up to 256: the heads of the group that share
 //    the kept blocks, BLK rows each -- form two M = 128 tiles whose Q stays
-//    in shared memory; every kept key block is walked as 64-token sub-tiles,
-//    so one K/V copy serves every head of the group;
+//    in shared memory. The kept key blocks are walked as 128-key sub-tiles
+//    (two kept 64-token blocks, or one 128-token block; the MMA does not care
+//    that the two halves are apart in the cache), so one K/V copy serves every
+//    head of the group and each MMA has N = 128;
 //  * warp 8, one lane: TMA producer (2-D tiles, 128-byte swizzle) of Q once
-//    and of K/V sub-tiles through a ring of stages;
-//  * warp 9, one lane: issues the MMAs. S_t = Q_t K^T (M 128, N 64, K D) into
-//    a double-buffered TMEM tile, then O_t += P_t V (M 128, N D, K 64) into a
-//    TMEM accumulator; the S of the next sub-tile is issued before the P V of
-//    this one, so the tensor core computes while the softmax runs;
-//  * warps 0-3 and 4-7: one softmax warpgroup per M tile, a thread per row
-//    (TMEM lane): reads S, masks (causal on the diagonal block, the sequence
-//    end), online softmax in the exp2 domain with a lazily moved reference
-//    maximum (O and l are rescaled in TMEM only when the row maximum grows by
-//    more than 2^8), writes P as bf16 into shared memory in the MMA's operand
-//    layout; at the end reads O, divides by l and stores the row;
+//    and of K and V through separate rings (K is released as soon as both S
+//    tiles have read it, V after both P V);
+//  * warp 9, one lane: issues the MMAs in the order P V_0(n), S_0(n+1),
+//    P V_1(n), S_1(n+1), so the tensor core computes one tile while the other
+//    tile's softmax runs. S_t = Q_t K^T (M 128, N 128, K D) lands in TMEM; the
+//    softmax writes P_t as bf16 over it; O_t += P_t V takes P_t straight from
+//    TMEM (A operand in tensor memory) -- no P round trip through shared
+//    memory, which would cost operand bandwidth;
+//  * warps 0-3 and 4-7: one softmax warpgroup per tile, a thread per row
+//    (TMEM lane): reads its S row, masks (causal on the diagonal block, the
+//    sequence end, an absent second half), online softmax in the exp2 domain
+//    with a lazily moved reference maximum (O and l are rescaled in TMEM only
+//    when the row maximum grows by more than 2^8), writes P; at the end reads
+//    O, divides by l and stores the row;
 //  * every wait is bounded; on expiry the CTA stops, drains its own copies and
 //    MMAs, frees its tensor memory and writes NaN rows.
 #include <cuda_bf16.h>
@@ -41,10 +46,11 @@ constexpr int kAttnThreads = 320;   // 8 softmax warps, producer, MMA
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kRowsPerCta = 256;    // two M = 128 tiles
-constexpr int kSub = 64;            // key tokens per sub-tile
-constexpr int kTmemCols = 512;
+constexpr int kHalf = 64;           // key tokens per half sub-tile (one TMA box of rows)
+constexpr int kSub = 128;           // key tokens per sub-tile
+constexpr int kTmemCols = 512;      // per tile: O at +0 (D columns), S at +128 (128 columns), P at +192
+constexpr int kSCol = 128;
 constexpr int kAttnSmemLimit = 232448;
-constexpr int kMaxAttnStages = 8;
 constexpr float kLog2eA = 1.44269504088896340736f;
 constexpr float kLn2A = 0.69314718055994530942f;
 constexpr float kRescaleLog2 = 8.0f;  // move the reference maximum only past a 2^8 growth
@@ -52,54 +58,57 @@ constexpr int kListCap = 384;         // kept lists up to this length are staged
 
 template <int D>
 struct AttnCfg {
-    static constexpr int kBoxes = D / 64;               // 128-byte column boxes of a row
-    static constexpr int kQTile = kBoxes * 128 * 128;   // one M tile of Q
-    static constexpr int kPTile = 128 * 128;            // one M tile of P (64 tokens)
-    static constexpr int kKV = kBoxes * kSub * 128;     // K (or V) of one sub-tile
-    static constexpr int kStage = 2 * kKV;
-    static constexpr int kFixed = 2 * kQTile + 2 * kPTile;
+    static constexpr int kBoxes = D / 64;                // 128-byte column boxes of a row
+    static constexpr int kQTile = kBoxes * 128 * 128;    // one M tile of Q
+    static constexpr int kBox = kSub * 128;              // one column box of a K or V sub-tile
+    static constexpr int kKV = kBoxes * kBox;            // K (or V) of one sub-tile
     static constexpr int kBarBytes = 256 + kListCap * 4;
-    static constexpr int kStages0 = (kAttnSmemLimit - 1024 - kBarBytes - kFixed) / kStage;
-    static constexpr int kStages = kStages0 > kMaxAttnStages ? kMaxAttnStages : kStages0;
-    static constexpr int kSmem = 1024 + kFixed + kStages * kStage + kBarBytes;
-    static constexpr int kOCol = 0;                     // per tile: O at +0, S buffers at +D, +D+64
-    static_assert(kStages >= 2, "too little shared memory for the K/V ring");
-    static_assert(D + 2 * kSub <= kTmemCols / 2, "TMEM columns of one tile");
+    static constexpr int kRing = (kAttnSmemLimit - 1024 - kBarBytes - 2 * kQTile) / kKV;  // K + V slots
+    static constexpr int kVSt = kRing / 2 > 4 ? 4 : kRing / 2;
+    static constexpr int kKSt = kRing - kVSt > 4 ? 4 : kRing - kVSt;
+    static constexpr int kSmem = 1024 + 2 * kQTile + (kKSt + kVSt) * kKV + kBarBytes;
+    static_assert(kVSt >= 2 && kKSt >= 2, "too little shared memory for the K/V rings");
+    static_assert(D <= kSCol && kSCol + kSub <= kTmemCols / 2, "TMEM columns of one tile");
 };
 
-// The kept (b, kvh, i) list walked as 64-token sub-tiles: entries outside
-// [0, i] are skipped, and so is a second half that starts at or past L.
-struct SubIter {
+// The kept (b, kvh, i) list walked as sub-tiles of two 64-token halves:
+// entries outside [0, i] are skipped; with 64-token blocks a sub-tile takes
+// two consecutive kept blocks (the last one may have one), with 128-token
+// blocks one block, its second half absent when it starts at or past L.
+struct PairIter {
     const int32_t* list;
-    int nsel, i, L, blk, halves;
-    int x, hh, j;
-    __device__ void seek() {
+    int nsel, i, L, blk;
+    int x;            // next list position
+    int tokA, tokB;   // token bases of the halves; tokB < 0: absent
+    bool valid;
+    __device__ int next_entry() {
         while (x < nsel) {
-            j = list[x];
-            if (j >= 0 && j <= i && j * blk + kSub * hh < L) return;
-            ++x;
-            hh = 0;
+            const int j = list[x++];
+            if (j >= 0 && j <= i && j * blk < L) return j;
+        }
+        return -1;
+    }
+    __device__ void advance() {
+        const int ja = next_entry();
+        valid = ja >= 0;
+        if (!valid) return;
+        tokA = ja * blk;
+        if (blk == kSub) {
+            tokB = tokA + kHalf < L ? tokA + kHalf : -1;
+        } else {
+            const int jb = next_entry();
+            tokB = jb >= 0 ? jb * blk : -1;
         }
     }
     __device__ void start() {
         x = 0;
-        hh = 0;
-        seek();
-    }
-    __device__ bool done() const { return x >= nsel; }
-    __device__ int tok0() const { return j * blk + kSub * hh; }
-    __device__ void next() {
-        if (++hh == halves) {
-            hh = 0;
-            ++x;
-        }
-        seek();
+        advance();
     }
 };
 
 struct AttnBars {
-    uint32_t q_full, kv_full, kv_empty, s_ready, s_free, p_ready, pv_done, drain;
-    // kv_full / kv_empty: + 8 * stage; s_ready / s_free: + 8 * (2 * tile + buffer); p_ready / pv_done: + 8 * tile
+    uint32_t q_full, k_full, k_empty, v_full, v_empty, s_ready, p_ready, o_done, drain;
+    // k_* : + 8 * slot, v_* : + 8 * slot; s_ready / p_ready / o_done: + 8 * tile
 };
 
 // 2^x on the special-function unit (flush-to-zero; 2^-inf = 0).
@@ -150,22 +159,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return;
     }
 
-    // ---- shared memory: Q tiles, P tiles, K/V stages, barriers
+    // ---- shared memory: Q tiles, K ring, V ring, barriers, kept list
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base, sP = base + 2 * C::kQTile, sKV = sP + 2 * C::kPTile;
-    const uint32_t sBar = sKV + C::kStages * C::kStage;
+    const uint32_t sQ = base, sK = base + 2 * C::kQTile, sV = sK + C::kKSt * C::kKV;
+    const uint32_t sBar = sV + C::kVSt * C::kKV;
     unsigned char* gBar = gbase + (sBar - base);
     AttnBars bars;
     bars.q_full = sBar;
-    bars.kv_full = sBar + 8;
-    bars.kv_empty = bars.kv_full + 8 * C::kStages;
-    bars.s_ready = bars.kv_empty + 8 * C::kStages;
-    bars.s_free = bars.s_ready + 8 * 4;
-    bars.p_ready = bars.s_free + 8 * 4;
-    bars.pv_done = bars.p_ready + 8 * 2;
-    bars.drain = bars.pv_done + 8 * 2;
+    bars.k_full = sBar + 8;
+    bars.k_empty = bars.k_full + 8 * C::kKSt;
+    bars.v_full = bars.k_empty + 8 * C::kKSt;
+    bars.v_empty = bars.v_full + 8 * C::kVSt;
+    bars.s_ready = bars.v_empty + 8 * C::kVSt;
+    bars.p_ready = bars.s_ready + 8 * 2;
+    bars.o_done = bars.p_ready + 8 * 2;
+    bars.drain = bars.o_done + 8 * 2;
     const uint32_t bar_end = bars.drain + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + (bar_end - sBar));
     int* abort_flag = reinterpret_cast<int*>(gBar + (bar_end - sBar) + 4);
@@ -173,17 +183,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (tid == 0) {
         mbar_init(bars.q_full, 1);
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(bars.kv_full + 8 * s, 1);
-            mbar_init(bars.kv_empty + 8 * s, 1);
+        for (int s = 0; s < C::kKSt; ++s) {
+            mbar_init(bars.k_full + 8 * s, 1);
+            mbar_init(bars.k_empty + 8 * s, 1);
         }
-        for (int x = 0; x < 4; ++x) {
-            mbar_init(bars.s_ready + 8 * x, 1);
-            mbar_init(bars.s_free + 8 * x, 4);
+        for (int s = 0; s < C::kVSt; ++s) {
+            mbar_init(bars.v_full + 8 * s, 1);
+            mbar_init(bars.v_empty + 8 * s, 1);
         }
         for (int t = 0; t < 2; ++t) {
+            mbar_init(bars.s_ready + 8 * t, 1);
             mbar_init(bars.p_ready + 8 * t, 4);
-            mbar_init(bars.pv_done + 8 * t, 1);
+            mbar_init(bars.o_done + 8 * t, 1);
         }
         mbar_init(bars.drain, 1);
         *abort_flag = 0;
@@ -202,15 +213,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-    SubIter it0;
+    PairIter it0;
     it0.list = list;
     it0.nsel = nsel;
     it0.i = i;
     it0.L = L;
     it0.blk = BLK;
-    it0.halves = BLK / kSub;
     it0.start();
-    const bool any = !it0.done();
+    const bool any = it0.valid;
 
     auto fail = [&]() { atomicExch(abort_flag, 1); };
 
@@ -231,32 +241,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // K/V tiles are re-read by the other query blocks of the row: keep them in L2
             uint64_t keep;
             asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
-            SubIter it = it0;
+            PairIter it = it0;
             int n = 0;
-            for (; !it.done(); it.next(), ++n) {
-                const int st = n % C::kStages;
-                if (n >= C::kStages && !mbar_wait(bars.kv_empty + 8 * st, (uint32_t)((n / C::kStages - 1) & 1))) {
-                    fail();
+            bool ok = true;
+            for (; it.valid; it.advance(), ++n) {
+                const int halves = it.tokB >= 0 ? 2 : 1;
+                const uint32_t bytes = (uint32_t)(halves * C::kBoxes * kHalf * 128);
+                const int ks = n % C::kKSt, vs = n % C::kVSt;
+                if (n >= C::kKSt && !mbar_wait(bars.k_empty + 8 * ks, (uint32_t)((n / C::kKSt - 1) & 1))) ok = false;
+                if (!ok || abort_set(abort_flag)) break;
+                mbar_arrive_expect_tx(bars.k_full + 8 * ks, bytes);
+                for (int h = 0; h < halves; ++h) {
+                    const int y = row * Lmax + (h == 0 ? it.tokA : it.tokB);
+                    for (int c = 0; c < C::kBoxes; ++c)
+                        tma_load_2d(sK + ks * C::kKV + c * C::kBox + h * kHalf * 128, &tmK, bars.k_full + 8 * ks,
+                                    c * 64, y, keep);
+                }
+                if (n >= C::kVSt && !mbar_wait(bars.v_empty + 8 * vs, (uint32_t)((n / C::kVSt - 1) & 1))) ok = false;
+                if (!ok || abort_set(abort_flag)) {
+                    ++n;  // the K copies of this sub-tile are in flight
                     break;
                 }
-                if (abort_set(abort_flag)) break;
-                const uint32_t stage = sKV + st * C::kStage;
-                const uint32_t bar = bars.kv_full + 8 * st;
-                mbar_arrive_expect_tx(bar, (uint32_t)C::kStage);
-                const int y = row * Lmax + it.tok0();
-                for (int c = 0; c < C::kBoxes; ++c) {
-                    tma_load_2d(stage + c * kSub * 128, &tmK, bar, c * 64, y, keep);
-                    tma_load_2d(stage + C::kKV + c * kSub * 128, &tmV, bar, c * 64, y, keep);
+                mbar_arrive_expect_tx(bars.v_full + 8 * vs, bytes);
+                for (int h = 0; h < halves; ++h) {
+                    const int y = row * Lmax + (h == 0 ? it.tokA : it.tokB);
+                    for (int c = 0; c < C::kBoxes; ++c)
+                        tma_load_2d(sV + vs * C::kKV + c * C::kBox + h * kHalf * 128, &tmV, bars.v_full + 8 * vs,
+                                    c * 64, y, keep);
                 }
             }
+            if (!ok) fail();
             // leave only after the copies issued have landed
             const int issued = n;
-            for (int m = max(0, issued - C::kStages); m < issued; ++m)
-                (void)mbar_wait(bars.kv_full + 8 * (m % C::kStages), (uint32_t)((m / C::kStages) & 1));
+            for (int m = max(0, issued - C::kKSt); m < issued; ++m)
+                (void)mbar_wait(bars.k_full + 8 * (m % C::kKSt), (uint32_t)((m / C::kKSt) & 1));
+            for (int m = max(0, issued - C::kVSt); m < issued; ++m)
+                (void)mbar_wait(bars.v_full + 8 * (m % C::kVSt), (uint32_t)((m / C::kVSt) & 1));
             (void)mbar_wait(bars.q_full, 0u);
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+    }
+    else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issue
         if (lane == 0 && any) {
             constexpr uint32_t kIdS = tc::idesc_bf16_f32(128, kSub, false);
@@ -264,40 +289,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             bool ok = mbar_wait(bars.q_full, 0u);
             const uint64_t dq0 = tc::smem_desc_sw128(sQ, 16, 1024);
             const uint64_t dq1 = tc::smem_desc_sw128(sQ + C::kQTile, 16, 1024);
-            const uint64_t dp0 = tc::smem_desc_sw128(sP, 16, 1024);
-            const uint64_t dp1 = tc::smem_desc_sw128(sP + C::kPTile, 16, 1024);
-            // S_t(n) = Q_t K(n)^T into buffer n % 2 of tile t
-            auto issue_s = [&](int n) -> bool {
-                const int st = n % C::kStages;
-                if (!mbar_wait(bars.kv_full + 8 * st, (uint32_t)((n / C::kStages) & 1))) return false;
-                const uint64_t dk = tc::smem_desc_sw128(sKV + st * C::kStage, 16, 1024);
-                for (int t = 0; t < n_tiles; ++t) {
-                    const int buf = n & 1;
-                    if (n >= 2 && !mbar_wait(bars.s_free + 8 * (2 * t + buf), (uint32_t)(((n - 2) >> 1) & 1)))
-                        return false;
-                    tc::fence_after_sync();
-                    const uint32_t d_tmem = tmem + (uint32_t)(t * (kTmemCols / 2) + D + buf * kSub);
-                    const uint64_t dq = t == 0 ? dq0 : dq1;
-                    // k-th 16-column step: box k / 4, 32 bytes * (k % 4) into the swizzled row
+            // S_t(n) = Q_t K(n)^T into the tile's S columns; the k-th 16-column step
+            // is box k / 4, 32 bytes * (k % 4) into each swizzled 128-byte row
+            auto issue_s = [&](int t, int n) {
+                const uint64_t dk = tc::smem_desc_sw128(sK + (n % C::kKSt) * C::kKV, 16, 1024);
+                const uint64_t dq = t == 0 ? dq0 : dq1;
+                const uint32_t d_tmem = tmem + (uint32_t)(t * (kTmemCols / 2) + kSCol);
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        tc::mma_bf16_ss(d_tmem, dq + (uint64_t)((k >> 2) * (128 * 128 / 16) + (k & 3) * 2),
-                                        dk + (uint64_t)((k >> 2) * (kSub * 128 / 16) + (k & 3) * 2), kIdS, k > 0);
-                    tc::commit(bars.s_ready + 8 * (2 * t + buf));
-                }
-                return true;
+                for (int k = 0; k < D / 16; ++k)
+                    tc::mma_bf16_ss(d_tmem, dq + (uint64_t)((k >> 2) * (128 * 128 / 16) + (k & 3) * 2),
+                                    dk + (uint64_t)((k >> 2) * (C::kBox / 16) + (k & 3) * 2), kIdS, k > 0);
+                tc::commit(bars.s_ready + 8 * t);
             };
-            SubIter it = it0;
+            if (ok) ok = mbar_wait(bars.k_full, 0u);  // K(0): slot 0, first phase
+            if (ok) {
+                tc::fence_after_sync();
+                for (int t = 0; t < n_tiles; ++t) issue_s(t, 0);
+                tc::commit(bars.k_empty);  // slot 0 is free once both S(0) are done
+            }
+            PairIter it = it0;
             int n = 0;
-            if (ok) ok = issue_s(0);
-            while (ok && !it.done()) {
-                SubIter nx = it;
-                nx.next();
-                if (!nx.done()) {
-                    ok = issue_s(n + 1);
-                    if (!ok) break;
+            while (ok && it.valid) {
+                PairIter nx = it;
+                nx.advance();
+                const bool more = nx.valid;
+                const int vs = n % C::kVSt, ks1 = (n + 1) % C::kKSt;
+                const int ksteps = it.tokB >= 0 ? kSub / 16 : kHalf / 16;  // an absent half is skipped
+                if (!mbar_wait(bars.v_full + 8 * vs, (uint32_t)((n / C::kVSt) & 1)) ||
+                    (more && !mbar_wait(bars.k_full + 8 * ks1, (uint32_t)(((n + 1) / C::kKSt) & 1)))) {
+                    ok = false;
+                    break;
                 }
-                const uint64_t dv = tc::smem_desc_sw128(sKV + (n % C::kStages) * C::kStage + C::kKV, kSub * 128, 1024);
+                // V: MN-major (keys x D); the k-th 16-key step is 16 rows further, the
+                // next 64 columns of D one box further (leading byte offset)
+                const uint64_t dv = tc::smem_desc_sw128(sV + vs * C::kKV, C::kBox, 1024);
                 for (int t = 0; t < n_tiles; ++t) {
                     if (!mbar_wait(bars.p_ready + 8 * t, (uint32_t)(n & 1))) {
                         ok = false;
@@ -305,16 +330,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                     tc::fence_after_sync();
                     const uint32_t o_tmem = tmem + (uint32_t)(t * (kTmemCols / 2));
-                    const uint64_t dp = t == 0 ? dp0 : dp1;
-                    // k-th 16-token step: 32 bytes into each P row, 16 V rows further
-#pragma unroll
-                    for (int k = 0; k < kSub / 16; ++k)
-                        tc::mma_bf16_ss(o_tmem, dp + (uint64_t)(k * 2), dv + (uint64_t)(k * (16 * 128 / 16)), kIdO,
-                                        n > 0 || k > 0);
-                    tc::commit(bars.pv_done + 8 * t);
+                    for (int k = 0; k < ksteps; ++k)
+                        tc::mma_bf16_ts(o_tmem, o_tmem + (uint32_t)(kSCol + 64 + k * 8),
+                                        dv + (uint64_t)(k * (16 * 128 / 16)), kIdO, n > 0 || k > 0);
+                    // S_t(n+1) overwrites P_t(n) only after P V_t(n) has read it: the tensor
+                    // core runs one thread's MMAs in issue order
+                    if (more) issue_s(t, n + 1);
                 }
                 if (!ok) break;
-                tc::commit(bars.kv_empty + 8 * (n % C::kStages));  // S(n) and P V(n) read the stage
+                tc::commit(bars.v_empty + 8 * vs);           // V(n) read by every P V
+                if (more) tc::commit(bars.k_empty + 8 * ks1);  // K(n+1) read by every S
                 if (abort_set(abort_flag)) {
                     ok = false;
                     break;
@@ -323,6 +348,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 ++n;
             }
             if (!ok) fail();
+            for (int t = 0; t < n_tiles; ++t) tc::commit(bars.o_done + 8 * t);
             // every MMA issued has completed before the tensor memory is freed
             tc::commit(bars.drain);
             (void)mbar_wait(bars.drain, 0u);
@@ -339,98 +365,119 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int lim_tok = min(qt, L - 1);          // last key token this row may see
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t t_tmem = tmem + lane_base + (uint32_t)(t * (kTmemCols / 2));
-        const uint32_t p_row = sP + t * C::kPTile + r * 128;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        SubIter it = it0;
+        PairIter it = it0;
         int n = 0;
-        for (; !it.done(); it.next(), ++n) {
-            const int buf = n & 1;
-            bool w = mbar_wait(bars.s_ready + 8 * (2 * t + buf), (uint32_t)((n >> 1) & 1));
+        for (; it.valid; it.advance(), ++n) {
+            const bool w = mbar_wait(bars.s_ready + 8 * t, (uint32_t)(n & 1));
             if (__any_sync(0xffffffffu, !w || abort_set(abort_flag))) {  // one decision for the warp
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            uint32_t s[2][32];
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(D + buf * kSub), s[0]);
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(D + buf * kSub + 32), s[1]);
+            // mask (only the diagonal, the sequence end, an absent half)
+            const int limA = lim_tok - it.tokA;
+            const int limB = it.tokB >= 0 ? lim_tok - it.tokB : -1;
+            const bool masked = !__all_sync(0xffffffffu, limA >= kHalf - 1 && limB >= kHalf - 1);
+            // half A (keys 0-63): its maximum only; half B (keys 64-127) stays in registers
+            uint32_t sh[2][32];
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sh[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sh[1]);
             tc::wait_ld();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bars.s_free + 8 * (2 * t + buf));
-            // mask (only the diagonal and the sequence end), then the row maximum of the raw scores
-            const int lim = lim_tok - it.tok0();   // columns 0 .. lim are visible
-            if (!__all_sync(0xffffffffu, lim >= kSub - 1)) {
+            float m8[8];
 #pragma unroll
-                for (int c = 0; c < kSub; ++c)
-                    if (c > lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+            for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kHalf; ++c)
+                if (!masked || c <= limA) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c >> 5][c & 31]));
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 64), sh[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 96), sh[1]);
+            tc::wait_ld();
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < kHalf; ++c)
+                    if (c > limB) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < kSub; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(s[c >> 5][c & 31]));
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * scale_log2;  // scale > 0
+            for (int c = 0; c < kHalf; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c >> 5][c & 31]));
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;  // scale > 0
             float alpha = 1.f;
             if (mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx > -INFINITY)) {
                 alpha = m_ref == -INFINITY ? 0.f : ex2(m_ref - mx);
                 m_ref = mx;
                 l *= alpha;
             }
+            // P = 2^(s * scale - m) as bf16 pairs over the upper 64 S columns (keys 64-127 read
+            // already): half B into columns +96.., then half A, read again, into +64..
             const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-            uint32_t pk[kSub / 2];
             float sum2[2] = {0.f, 0.f};
+            auto emit = [&](int col) {
 #pragma unroll
-            for (int c = 0; c < kSub; c += 2) {
-                const float p0 = ex2(fmaf(__uint_as_float(s[c >> 5][c & 31]), scale_log2, neg_m));
-                const float p1 = ex2(fmaf(__uint_as_float(s[(c + 1) >> 5][(c + 1) & 31]), scale_log2, neg_m));
-                sum2[(c >> 1) & 1] += p0 + p1;
-                pk[c / 2] = pack_bf16x2(p0, p1);
-            }
-            l += sum2[0] + sum2[1];
-            // P and O are free once the previous P V has completed
-            if (n > 0) {
-                w = mbar_wait(bars.pv_done + 8 * t, (uint32_t)((n - 1) & 1));
-                if (__any_sync(0xffffffffu, !w)) {
-                    ok = false;
-                    break;
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sh[q][2 * e]), scale_log2, neg_m));
+                        const float p1 = ex2(fmaf(__uint_as_float(sh[q][2 * e + 1]), scale_log2, neg_m));
+                        sum2[e & 1] += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tc::st_32x32b_x16(t_tmem + (uint32_t)(col + 16 * q), pk);
                 }
-                tc::fence_after_sync();
-            }
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + ((ch ^ (r & 7)) << 4)),
-                             "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
-                             : "memory");
+            };
+            emit(kSCol + 96);
+            // O_t is final up to P V_t(n-1) (issued before S_t(n)): rescale it if needed
             if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t o[32];
-                    tc::ld_32x32b_x32(t_tmem + (uint32_t)(C::kOCol + c0), o);
+                    tc::ld_32x32b_x32(t_tmem + (uint32_t)c0, o);
                     tc::wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tc::st_32x32b_x32(t_tmem + (uint32_t)(C::kOCol + c0), o);
-                }
-                tc::wait_st();
-            }
-            // the sequence end inside this sub-tile: zero the V rows past it (they may hold anything)
-            if (t == 0 && it.tok0() + kSub > L) {
-                const int v0 = L - it.tok0();
-                const uint32_t sv = sKV + (n % C::kStages) * C::kStage + C::kKV;
-                for (int x = (warp & 3) * 32 + lane; x < (kSub - v0) * C::kBoxes * 8; x += 128) {
-                    const int rr = v0 + x / (C::kBoxes * 8), rem = x % (C::kBoxes * 8);
-                    const uint32_t a = sv + (rem >> 3) * (kSub * 128) + rr * 128 + (rem & 7) * 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                    tc::st_32x32b_x32(t_tmem + (uint32_t)c0, o);
                 }
             }
-            fence_proxy_async_smem();
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sh[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sh[1]);
+            tc::wait_ld();
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < kHalf; ++c)
+                    if (c > limA) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+            }
+            emit(kSCol + 64);
+            l += sum2[0] + sum2[1];
+            tc::wait_st();
+            // the sequence end inside a half: zero its V rows past L (they may hold anything)
+            if (t == 0) {
+                const int vA = it.tokA + kHalf > L ? L - it.tokA : kHalf;
+                const int vB = it.tokB >= 0 && it.tokB + kHalf > L ? L - it.tokB : kHalf;
+                if (vA < kHalf || vB < kHalf) {
+                    const int vs = n % C::kVSt;
+                    const bool wv = mbar_wait(bars.v_full + 8 * vs, (uint32_t)((n / C::kVSt) & 1));
+                    if (!wv) fail();
+                    const uint32_t sv = sV + vs * C::kKV;
+                    for (int h = 0; h < 2; ++h) {
+                        const int v0 = h == 0 ? vA : vB;
+                        for (int x = (warp & 3) * 32 + lane; x < (kHalf - v0) * C::kBoxes * 8; x += 128) {
+                            const int rr = h * kHalf + v0 + x / (C::kBoxes * 8), rem = x % (C::kBoxes * 8);
+                            const uint32_t a = sv + (rem >> 3) * C::kBox + rr * 128 + (rem & 7) * 16;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                        }
+                    }
+                    fence_proxy_async_smem();
+                }
+            }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.p_ready + 8 * t);
         }
         // ---- epilogue: O / l
-        if (ok && n > 0) {
-            const bool w = mbar_wait(bars.pv_done + 8 * t, (uint32_t)((n - 1) & 1));
+        if (ok) {
+            const bool w = mbar_wait(bars.o_done + 8 * t, 0u);
             if (__any_sync(0xffffffffu, !w)) ok = false;
             tc::fence_after_sync();
         }
@@ -443,7 +490,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(C::kOCol + c0), o);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)c0, o);
             tc::wait_ld();
             if (write) {
                 uint32_t pkd[16];
