@@ -64,8 +64,10 @@ struct AttnCfg {
     static constexpr int kKV = kBoxes * kBox;            // K (or V) of one sub-tile
     static constexpr int kBarBytes = 256 + kListCap * 4;
     static constexpr int kRing = (kAttnSmemLimit - 1024 - kBarBytes - 2 * kQTile) / kKV;  // K + V slots
-    static constexpr int kVSt = kRing / 2 > 4 ? 4 : kRing / 2;
-    static constexpr int kKSt = kRing - kVSt > 4 ? 4 : kRing - kVSt;
+    // a V slot is held from its copy until both P V have read it, a K slot only
+    // until both S have: V gets the deeper ring
+    static constexpr int kKSt = kRing >= 8 ? 4 : 2;
+    static constexpr int kVSt = kRing - kKSt > 6 ? 6 : kRing - kKSt;
     static constexpr int kSmem = 1024 + 2 * kQTile + (kKSt + kVSt) * kKV + kBarBytes;
     static_assert(kVSt >= 2 && kKSt >= 2, "too little shared memory for the K/V rings");
     static_assert(D <= kSCol && kSCol + kSub <= kTmemCols / 2, "TMEM columns of one tile");
@@ -116,6 +118,24 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// P for 64 scores of a row: 2^(s * scale + neg_m) as bf16 pairs into 32 TMEM
+// columns from `taddr`; the row sum goes to sum2.
+__device__ __forceinline__ void emit_p(const uint32_t (&sh)[2][32], float scale_log2, float neg_m, float (&sum2)[2],
+                                       uint32_t taddr) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(sh[q][2 * e]), scale_log2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(sh[q][2 * e + 1]), scale_log2, neg_m));
+            sum2[e & 1] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+        }
+        tc::st_32x32b_x16(taddr + (uint32_t)(16 * q), pk);
+    }
 }
 
 __device__ __forceinline__ bool abort_set(const int* flag) { return *(volatile const int*)flag != 0; }
@@ -380,27 +400,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int limA = lim_tok - it.tokA;
             const int limB = it.tokB >= 0 ? lim_tok - it.tokB : -1;
             const bool masked = !__all_sync(0xffffffffu, limA >= kHalf - 1 && limB >= kHalf - 1);
-            // half A (keys 0-63): its maximum only; half B (keys 64-127) stays in registers
-            uint32_t sh[2][32];
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sh[0]);
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sh[1]);
-            tc::wait_ld();
-            float m8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < kHalf; ++c)
-                if (!masked || c <= limA) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c >> 5][c & 31]));
+            // the whole S row: four loads in flight, one wait
+            uint32_t sa[2][32], sh[2][32];
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sa[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sa[1]);
             tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 64), sh[0]);
             tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 96), sh[1]);
             tc::wait_ld();
             if (masked) {
 #pragma unroll
-                for (int c = 0; c < kHalf; ++c)
+                for (int c = 0; c < kHalf; ++c) {
+                    if (c > limA) sa[c >> 5][c & 31] = __float_as_uint(-INFINITY);
                     if (c > limB) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                }
             }
+            float m8[8];
 #pragma unroll
-            for (int c = 0; c < kHalf; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c >> 5][c & 31]));
+            for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kHalf; ++c) {
+                m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sa[c >> 5][c & 31]));
+                m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c >> 5][c & 31]));
+            }
             const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;  // scale > 0
             float alpha = 1.f;
@@ -409,25 +430,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 m_ref = mx;
                 l *= alpha;
             }
-            // P = 2^(s * scale - m) as bf16 pairs over the upper 64 S columns (keys 64-127 read
-            // already): half B into columns +96.., then half A, read again, into +64..
+            // P = 2^(s * scale - m) as bf16 pairs over the upper 64 S columns (every S column is
+            // in registers by now): keys 64-127 into columns +96.., keys 0-63 into +64..
             const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
             float sum2[2] = {0.f, 0.f};
-            auto emit = [&](int col) {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sh[q][2 * e]), scale_log2, neg_m));
-                        const float p1 = ex2(fmaf(__uint_as_float(sh[q][2 * e + 1]), scale_log2, neg_m));
-                        sum2[e & 1] += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-                    tc::st_32x32b_x16(t_tmem + (uint32_t)(col + 16 * q), pk);
-                }
-            };
-            emit(kSCol + 96);
+            emit_p(sh, scale_log2, neg_m, sum2, t_tmem + (uint32_t)(kSCol + 96));
+            emit_p(sa, scale_log2, neg_m, sum2, t_tmem + (uint32_t)(kSCol + 64));
             // O_t is final up to P V_t(n-1) (issued before S_t(n)): rescale it if needed
             if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -440,15 +448,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tc::st_32x32b_x32(t_tmem + (uint32_t)c0, o);
                 }
             }
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sh[0]);
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sh[1]);
-            tc::wait_ld();
-            if (masked) {
-#pragma unroll
-                for (int c = 0; c < kHalf; ++c)
-                    if (c > limA) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-            }
-            emit(kSCol + 64);
             l += sum2[0] + sum2[1];
             tc::wait_st();
             // the sequence end inside a half: zero its V rows past L (they may hold anything)
