@@ -120,19 +120,28 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // P for 64 scores of a row: 2^(s * scale + neg_m) as bf16 pairs into 32 TMEM
-// columns from `taddr`; the row sum goes to sum2.
-__device__ __forceinline__ void emit_p(const uint32_t (&sh)[2][32], float scale_log2, float neg_m, float (&sum2)[2],
+// columns from `taddr` (paired fp32 FMA and add); the row sum goes to sum2.
+__device__ __forceinline__ void emit_p(const uint32_t (&sh)[2][32], float scale_log2, float neg_m, float2 (&sum2)[2],
                                        uint32_t taddr) {
+    const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(neg_m, neg_m);
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(sh[q][2 * e]), scale_log2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(sh[q][2 * e + 1]), scale_log2, neg_m));
-            sum2[e & 1] += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sh[q][2 * e]), __uint_as_float(sh[q][2 * e + 1])),
+                                        sc, nm);
+            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+            sum2[e & 1] = __fadd2_rn(sum2[e & 1], pp);
+            pk[e] = pack_bf16x2(pp.x, pp.y);
         }
         tc::st_32x32b_x16(taddr + (uint32_t)(16 * q), pk);
     }
@@ -400,28 +409,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int limA = lim_tok - it.tokA;
             const int limB = it.tokB >= 0 ? lim_tok - it.tokB : -1;
             const bool masked = !__all_sync(0xffffffffu, limA >= kHalf - 1 && limB >= kHalf - 1);
-            // the whole S row: four loads in flight, one wait
-            uint32_t sa[2][32], sh[2][32];
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sa[0]);
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sa[1]);
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 64), sh[0]);
-            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 96), sh[1]);
+            // half A (keys 0-63): its maximum only; half B (keys 64-127) stays in registers
+            uint32_t sh[2][32];
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sh[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sh[1]);
             tc::wait_ld();
             if (masked) {
 #pragma unroll
-                for (int c = 0; c < kHalf; ++c) {
-                    if (c > limA) sa[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-                    if (c > limB) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-                }
+                for (int c = 0; c < kHalf; ++c)
+                    if (c > limA) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
             float m8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kHalf; ++c) {
-                m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sa[c >> 5][c & 31]));
-                m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c >> 5][c & 31]));
+            for (int c = 0; c < kHalf; c += 2)
+                m8[(c >> 1) & 7] = fmax3f(m8[(c >> 1) & 7], __uint_as_float(sh[c >> 5][c & 31]),
+                                          __uint_as_float(sh[c >> 5][(c + 1) & 31]));
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 64), sh[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 96), sh[1]);
+            tc::wait_ld();
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < kHalf; ++c)
+                    if (c > limB) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
+#pragma unroll
+            for (int c = 0; c < kHalf; c += 2)
+                m8[(c >> 1) & 7] = fmax3f(m8[(c >> 1) & 7], __uint_as_float(sh[c >> 5][c & 31]),
+                                          __uint_as_float(sh[c >> 5][(c + 1) & 31]));
             const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;  // scale > 0
             float alpha = 1.f;
@@ -430,12 +446,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 m_ref = mx;
                 l *= alpha;
             }
-            // P = 2^(s * scale - m) as bf16 pairs over the upper 64 S columns (every S column is
-            // in registers by now): keys 64-127 into columns +96.., keys 0-63 into +64..
+            // P = 2^(s * scale - m) as bf16 pairs over the upper 64 S columns (keys 64-127 read
+            // already): half B into columns +96.., then half A, read again, into +64..
             const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-            float sum2[2] = {0.f, 0.f};
-            emit_p(sh, scale_log2, neg_m, sum2, t_tmem + (uint32_t)(kSCol + 96));
-            emit_p(sa, scale_log2, neg_m, sum2, t_tmem + (uint32_t)(kSCol + 64));
+            float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            auto emit = [&](int col) { emit_p(sh, scale_log2, neg_m, sum2, t_tmem + (uint32_t)col); };
+            emit(kSCol + 96);
             // O_t is final up to P V_t(n-1) (issued before S_t(n)): rescale it if needed
             if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -448,7 +464,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tc::st_32x32b_x32(t_tmem + (uint32_t)c0, o);
                 }
             }
-            l += sum2[0] + sum2[1];
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)kSCol, sh[0]);
+            tc::ld_32x32b_x32(t_tmem + (uint32_t)(kSCol + 32), sh[1]);
+            tc::wait_ld();
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < kHalf; ++c)
+                    if (c > limA) sh[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+            }
+            emit(kSCol + 64);
+            l += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
             tc::wait_st();
             // the sequence end inside a half: zero its V rows past L (they may hold anything)
             if (t == 0) {
