@@ -1147,7 +1147,10 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     f.n_gate_stages = n_gate > kMaxGateStages ? kMaxGateStages : n_gate;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(num_sms, 1, 1);  // every SM: phase 1 spreads rows over all of them
+    // With one CTA per row in both phases nothing crosses CTAs: a plain launch of
+    // one CTA per row. Otherwise every SM, co-resident for the grid barrier.
+    const bool barrier = !(f.gate_ctas == f.rows && P == f.rows);
+    cfg.gridDim = dim3(barrier ? num_sms : f.rows, 1, 1);
     cfg.blockDim = dim3(kStepThreads, 1, 1);
     cfg.dynamicSmemBytes = l.total;
     cfg.stream = stream;
@@ -1155,7 +1158,7 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = barrier ? 1 : 0;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_step_kernel<D, BLK, DG>, tmK, tmV, p, f);
     if (e != cudaSuccess) (void)cudaGetLastError();  // a rejected launch must not leak into the next call
     return e;
