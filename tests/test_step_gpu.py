@@ -96,6 +96,24 @@ def test_fused_repeated_calls_reuse_workspace():
     assert api.seer_decode_wait_failures() == 0
 
 
+def test_fused_one_cta_per_row_needs_no_barrier():
+    # 80 rows on a 148-SM part: one CTA per row in both phases, a plain launch of 80
+    # CTAs; the grid barrier's counter is never touched
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rows = sms // 2 + 6
+    wl = W.Workload("rows", rows // 2, 8, 2, 128, 128, 64, 1024, 256)
+    lens = np.array([1024 - 7 * b for b in range(wl.batch)], np.int32)
+    inp = to_dev(W.make_inputs(wl, seed=21, pad_value=float("nan"), seq_lens=lens))
+    check_step(wl, inp)
+    st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
+    st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
+    for _ in range(3):
+        st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+    torch.cuda.synchronize()
+    assert int(st.workspace()[:8].view(torch.int64).item()) == 0
+    assert api.seer_decode_wait_failures() == 0
+
+
 @pytest.mark.parametrize("name,batches", [
     ("decode_b16", [0, 15]),
     ("large_block", [3]),
