@@ -112,6 +112,27 @@ def test_append_kv_validates_on_host():
     assert L.seer_append_kv(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, None) == api.SEER_ERR_UNSUPPORTED
 
 
+def test_prefill_validates_on_host():
+    d = _dims()
+    L = api.LIB
+    bad, unsup = api.SEER_ERR_INVALID_ARG, api.SEER_ERR_UNSUPPORTED
+    assert L.seer_prefill_gate_scores(None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == bad
+    assert L.seer_prefill_gate_scores(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, None) == bad
+    assert L.seer_prefill_select_blocks(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, None) == bad  # not k * blk
+    assert L.seer_prefill_select_blocks(ctypes.byref(d), FAKE, FAKE, 0, FAKE, FAKE, None) == bad
+    attn = L.seer_prefill_attention
+    assert attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0.0, FAKE, None, None) == bad  # kmax < 1
+    assert attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0.0, None, None, None) == bad  # no out
+    assert attn(ctypes.byref(d), FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0.0, FAKE, None, None) == bad  # q
+    assert attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0.0, FAKE + 8, None, None) == bad  # out
+    assert attn(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, float("nan"), FAKE, None, None) == bad
+    many_blocks = _dims(max_seq_len=4097 * 64)  # more than 4096 query blocks
+    assert attn(ctypes.byref(many_blocks), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0.0, FAKE, None, None) == unsup
+    # 4096 blocks, but 128 x 64 query rows of 262144 tokens do not fit a 32-bit TMA row coordinate
+    wide = _dims(batch=128, num_q_heads=64, num_kv_heads=8, max_seq_len=4096 * 64)
+    assert attn(ctypes.byref(wide), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0.0, FAKE, None, None) == unsup
+
+
 def test_python_wrapper_raises_on_error():
     with pytest.raises(api.SeerError) as e:
         api.seer_combine(_dims(head_dim=96), FAKE, FAKE, 4, FAKE, None, stream=0)
