@@ -20,15 +20,17 @@
 //  * warp 9, one lane: issues the MMAs in the order P V_0(n), S_0(n+1),
 //    P V_1(n), S_1(n+1), so the tensor core computes one tile while the other
 //    tile's softmax runs. S_t = Q_t K^T (M 128, N 128, K D) lands in TMEM; the
-//    softmax writes P_t as bf16 over it; O_t += P_t V takes P_t straight from
+//    softmax writes P_t as bf16 pairs over the upper 64 of its 128 columns
+//    (already read into registers); O_t += P_t V takes P_t straight from
 //    TMEM (A operand in tensor memory) -- no P round trip through shared
 //    memory, which would cost operand bandwidth;
 //  * warps 0-3 and 4-7: one softmax warpgroup per tile, a thread per row
 //    (TMEM lane): reads its S row, masks (causal on the diagonal block, the
 //    sequence end, an absent second half), online softmax in the exp2 domain
 //    with a lazily moved reference maximum (O and l are rescaled in TMEM only
-//    when the row maximum grows by more than 2^8), writes P; at the end reads
-//    O, divides by l and stores the row;
+//    when the row maximum grows by more than 2^8; the max is three-input
+//    max.f32, the scale-subtract and the row sum paired fp32 instructions),
+//    writes P; at the end reads O, divides by l and stores the row;
 //  * every wait is bounded; on expiry the CTA stops, drains its own copies and
 //    MMAs, frees its tensor memory and writes NaN rows.
 #include <cuda_bf16.h>
