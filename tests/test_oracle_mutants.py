@@ -52,6 +52,8 @@ MUTANTS = {
     "threshold_strict": [("if (s[j] >= threshold)", "if (s[j] > threshold)")],
     "prefill_not_causal": [("for (int u = j * blk; u < (j + 1) * blk && u <= t && u < L; ++u) tok[n++] = u;",
                             "for (int u = j * blk; u < (j + 1) * blk && u < L; ++u) tok[n++] = u;")],
+    "prefill_w_q_transposed": [("acc += qbar[d] * (double)W[(size_t)e * D + d];",
+                                "acc += qbar[d] * (double)W[(size_t)d * dg + e];")],
     "prefill_query_pool_summed": [("qbar[d] = acc / (double)(t1 - t0);", "qbar[d] = acc;")],
     "prefill_diagonal_not_forced": [("            out[n] = i;\n            *ns = n + 1;",
                                      "            out[n] = (i > 0 && n > 0) ? out[n - 1] : i;\n            *ns = n + 1;")],

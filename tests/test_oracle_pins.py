@@ -518,6 +518,26 @@ def test_prefill_gate_identity_weights_closed_form(oracle):
         assert np.all(np.isnan(s[b, :, NB:]))
 
 
+def test_prefill_toy_gate_matches_hand_derivation(oracle):
+    # Non-square, non-symmetric W_q (dg = 2, D = 4): a transposed or mis-strided
+    # projection changes every score of this example.
+    g = json.load(open(os.path.join(GOLDEN, "toy_prefill_gate.json")))
+    dm = g["dims"]
+    K = bits(np.array(g["K"], np.float32))[None, None]             # [1,1,6,4]
+    q = bits(np.array(g["q"], np.float32))[None]                   # [1,2,6,4]
+    wk = np.array(g["W_k"], np.float32)[None]
+    wq = np.array(g["W_q"], np.float32)[None]
+    lens = np.array([g["seq_len"]], np.int32)
+    kp = oracle.pool_project(K, wk, lens, dm["block_size"])
+    s = oracle.prefill_gate(q, wq, kp, lens, dm["block_size"])
+    expect = np.array([[np.nan if x is None else x for x in row] for row in g["scores"]])
+    np.testing.assert_allclose(s[0, 0], expect, rtol=0, atol=1e-13)  # NaN where j > i
+    for budget, lists in g["selection"].items():
+        idx, ns = oracle.prefill_select(s, lens, dm["block_size"], dm["max_seq_len"], int(budget))
+        for i, want in enumerate(lists):
+            assert list(idx[0, 0, i, :ns[0, 0, i]]) == want
+
+
 def test_prefill_selection_is_decode_selection_per_query_block(oracle):
     c = prefill_case(1, Lmax=64 * 12, lens=(64 * 12, 64 * 7 + 3))
     kp = oracle.pool_project(c["k"], c["w_k"], c["lens"], c["blk"])
