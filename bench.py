@@ -64,6 +64,8 @@ def parse():
     p.add_argument("--variant-steps", type=int, default=30, help="timed calls of each gate variant (0: skip)")
     p.add_argument("--prefill-steps", type=int, default=3, help="timed block-sparse prefills (0: skip)")
     p.add_argument("--prefill-batch", type=int, default=4, help="sequences of the prefill measurement")
+    p.add_argument("--config-steps", type=int, default=100,
+                   help="timed fused steps of each other decode workload (large block, ragged, sweep; 0: skip)")
     return p.parse_args()
 
 
@@ -302,6 +304,83 @@ def run_reference(args):
     print(json.dumps(line))
     del torch
     return 0
+
+
+# ---------------------------------------------------------------- the other decode workloads
+
+SWEEP = [f"sweep_b{b}_keep{k}" for b in (1, 4) for k in ("50", "30", "10", "05")]
+OTHER_WORKLOADS = ["large_block", "ragged"] + SWEEP
+
+
+def other_configs(args, dev, world, peak, flush, stream):
+    """The fused step on every other decode workload of the benchmark (same timing method as the
+    headline), each with its algorithmic bytes and roofline fraction; each sweep batch also gets this
+    build's dense decode (sparse decode + combine over every block) beside it."""
+    import torch
+
+    from block_sparse_attention_seer_b200 import api
+    from block_sparse_attention_seer_b200 import workloads as W
+
+    def timed(fn, n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for k in range(n + 5):
+            flush.zero_()
+            torch.cuda._sleep(300_000)
+            e = evs[k - 5] if k >= 5 else None
+            if e:
+                e[0].record(stream)
+            fn()
+            if e:
+                e[1].record(stream)
+        torch.cuda.synchronize()
+        us = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3
+        return max_over_ranks([us], dev)[0] if world > 1 else us
+
+    out = {}
+    rank = int(os.environ.get("RANK", "0"))
+    for name in OTHER_WORKLOADS + ["sweep_b1_dense", "sweep_b4_dense"]:
+        wl = W.WORKLOADS[name]
+        inp = W.make_inputs(wl, seed=args.seed + rank, device=dev)
+        lens = inp["seq_lens_host"]
+        entry = {"kept_fraction_target": None}
+        if not name.endswith("_dense"):
+            st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
+            st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
+            us = timed(lambda: st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"],
+                                             inp["seq_lens"]), args.config_steps)
+            step_bytes, _, toks, blocks = algorithmic_bytes(wl, lens, st.block_idx.cpu().numpy(),
+                                                            st.num_selected.cpu().numpy())
+            entry = {"us": round(us, 3), "bytes": step_bytes, "kept_blocks": blocks,
+                     "sparsity": round(1 - toks / float(sum(int(x) for x in lens) * wl.num_kv_heads), 4),
+                     "gbs": round(step_bytes / (us * 1e-6) / 1e9, 1),
+                     "frac": round(step_bytes / (us * 1e-6) / 1e9 / peak, 4),
+                     "frac_of_8tbs": round(step_bytes / (us * 1e-6) / 8e12, 4),
+                     "kernel": "decode_step_kernel (the whole step)"}
+            del st
+        else:  # this build's dense flash-decode at all blocks selected
+            st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
+            nbm = wl.nb_max
+            idx_d, ns_d = W.identity_block_list(lens, wl.num_kv_heads, wl.block_size, nbm)
+            idx_d = torch.from_numpy(idx_d).to(dev)
+            ns_d = torch.from_numpy(ns_d).to(dev)
+            us = timed(lambda: st.attend(inp["q"], inp["k_cache"], inp["v_cache"], inp["seq_lens"], idx_d, ns_d,
+                                         nbm), max(10, args.config_steps // 4))
+            _, dense_bytes, toks, _ = algorithmic_bytes(wl, lens, idx_d.cpu().numpy(), ns_d.cpu().numpy())
+            entry = {"us": round(us, 3), "bytes": dense_bytes, "gbs": round(dense_bytes / (us * 1e-6) / 1e9, 1),
+                     "frac": round(dense_bytes / (us * 1e-6) / 1e9 / peak, 4),
+                     "kernel": "sparse_decode + combine over every block (no gate)"}
+            del st, idx_d, ns_d
+        entry["description"] = wl.description
+        out[name] = entry
+        del inp
+        torch.cuda.empty_cache()
+    for b in (1, 4):  # each sweep point against the dense decode of its batch
+        d = out.get(f"sweep_b{b}_dense")
+        for k in ("50", "30", "10", "05"):
+            e = out.get(f"sweep_b{b}_keep{k}")
+            if d and e:
+                e["speedup_vs_dense"] = round(d["us"] / e["us"], 3)
+    return out
 
 
 # ---------------------------------------------------------------- our arm
@@ -600,6 +679,10 @@ def run_ours(args):
                "d2h_bytes_per_step": int(d2h),
                "path": "one packed H2D (q, new K, new V) -> seer_append_kv -> seer_decode_step -> D2H of out"}
 
+    configs = None
+    if args.config_steps > 0:
+        configs = other_configs(args, dev, world, peak, flush, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         us, cores, desc = oracle_sample_time(wl, host_inputs(inp), args.cpu_seconds)
@@ -629,6 +712,7 @@ def run_ours(args):
             "block_mass": block_mass,
             "gate_variants": variants,
             "prefill": prefill,
+            "other_workloads": configs,
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -177,6 +177,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // candidate i is kept iff key_i > kT, or key_i == kT and i <= iT.
 
 constexpr int kSelectBins = 2048;
+constexpr int kSelectHead = 32;  // list entries select_row can also leave in shared memory
 constexpr int kSelectBucket = 64;  // boundary bins up to this size are ranked exactly
 
 template <int kThreads>
@@ -236,8 +237,10 @@ struct SelectBins {
 // of the candidate blocks 0 .. NB-2. Writes the kept indices in ascending
 // order to out[0 .. kb-1] (kb = min(kmax, NB): block NB-1 always, plus the
 // kb-1 largest keys, equal keys going to the lower index) and -1 to out[kb ..
-// kmax). Every thread of the CTA calls it; shared memory is reused only after
-// a barrier that follows the call.
+// kmax). When `head` is given (shared memory, kSelectHead entries), the first
+// kSelectHead entries of the list are written there too. Every thread of the
+// CTA calls it; shared memory is reused only after a barrier that follows the
+// call.
 //
 // T is found by narrowing a key range [lo, hi] known to hold it: a histogram
 // of the range (SelectBins), a CTA scan of the bins from the top to the bin
@@ -246,24 +249,29 @@ struct SelectBins {
 // smallest and largest key. Every step removes at least one distinct key; a
 // range of one key value keeps its lowest indices. The common case is a
 // single histogram and seven barriers.
+
 template <int kThreads>
 __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __restrict__ out,
-                           SelectSmem<kThreads>& sm) {
+                           SelectSmem<kThreads>& sm, int32_t* head = nullptr) {
     constexpr int kWarps = kThreads / 32;
     constexpr unsigned kFull = 0xffffffffu;
     constexpr int kBinsPer = (kSelectBins + kThreads - 1) / kThreads;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto put = [&](int p, int v) {
+        out[p] = v;
+        if (head && p < kSelectHead) head[p] = v;
+    };
     const int kb = kmax < NB ? kmax : NB;
-    for (int p = (kb > 0 ? kb : 0) + tid; p < kmax; p += kThreads) out[p] = -1;
+    for (int p = (kb > 0 ? kb : 0) + tid; p < kmax; p += kThreads) put(p, -1);
     if (NB == 0) return;
     const int ncand = NB - 1;
     const int m = kb - 1;
     if (m >= ncand) {
-        for (int j = tid; j < NB; j += kThreads) out[j] = j;
+        for (int j = tid; j < NB; j += kThreads) put(j, j);
         return;
     }
     if (m == 0) {
-        if (tid == 0) out[0] = NB - 1;
+        if (tid == 0) put(0, NB - 1);
         return;
     }
     // Thread t owns the bins kSelectBins-1 - (t*kBinsPer + q), q < kBinsPer (from the top),
@@ -414,8 +422,8 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
     int pos = block_scan(n_sel, total);
     if (n_sel > 0)
         for (int i = c0; i < c1; ++i)
-            if (kept(i)) out[pos++] = i;
-    if (tid == 0) out[m] = NB - 1;
+            if (kept(i)) put(pos++, i);
+    if (tid == 0) put(m, NB - 1);
 }
 
 }  // namespace seer

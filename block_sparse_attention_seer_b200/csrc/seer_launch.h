@@ -60,9 +60,12 @@ struct StepLaunch {
     void* workspace;
 };
 
-// Byte offsets inside the step's workspace.
+// Byte offsets inside the step's workspace: the launch counter, the two
+// tallies of fully taken rows, per-row gate counts and decode states (all
+// zero before the first call: [0, counters_end)), then the gate's order keys
+// and the decode's partial slots.
 struct WorkspaceLayout {
-    size_t grid_bar, row_done, row_cnt, qg_flag, counters_end, qg, keys, o_part, lse_part, total;
+    size_t launch_ctr, rows_taken, row_cnt, row_state, counters_end, keys, o_part, lse_part, total;
 };
 WorkspaceLayout step_workspace_layout(const Shape& s, int kmax, int num_sms);
 

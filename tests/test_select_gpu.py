@@ -1,10 +1,13 @@
 """seer_select_blocks on adversarial scores: the kept lists must equal the
 oracle's selection on the same fp32 scores (widened exactly to fp64) bit for
-bit -- including all-equal scores (lowest indices win), clusters that share
-high-order bits (more radix passes), duplicated values at the boundary and
-signed zeros. Rows of up to 1024 candidates go through the single-warp
-select (16 candidates per lane up to 512, 32 above), longer ones through the
-CTA-wide radix select: the sizes straddle both switches."""
+bit -- including all-equal scores (lowest indices win), clusters within a few
+ulps (the value histogram narrows its key range over several steps), few
+distinct values, duplicated values at the boundary and signed zeros. The
+select (select_row) builds a histogram of the candidates' order keys over
+their value range, scans it from the top to the bin that holds the last
+kept key, ranks that bin exactly when it is small and narrows the range to
+it otherwise; the sizes run from 1 to 4096 candidates.
+"""
 import numpy as np
 import pytest
 import torch
@@ -48,7 +51,8 @@ CASES = {
 @pytest.mark.parametrize("case", sorted(CASES))
 @pytest.mark.parametrize("nb,blk,budget_blocks", [(2, 64, 1), (33, 64, 8), (512, 64, 64), (513, 64, 100),
                                                   (514, 64, 100), (1024, 128, 103), (1025, 64, 300),
-                                                  (1026, 64, 700), (4097, 64, 512)])
+                                                  (1026, 64, 700), (2049, 64, 300), (2050, 64, 1000),
+                                                  (4097, 64, 512)])
 def test_select_matches_oracle(case, nb, blk, budget_blocks):
     rng = np.random.default_rng(nb * 7 + len(case))
     B, Hkv = 2, 3

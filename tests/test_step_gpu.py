@@ -6,9 +6,12 @@ and against the separate five-call path.
 * refreshed pooled keys: identical to seer_kpool_update's;
 * output: within the attention tolerance of the fp64 oracle given the same
   block list, and of the five-call path;
-* repeated calls on one workspace give identical results (the in-kernel
-  row counters reset themselves; the grid barrier's arrival counter grows by
-  one grid per call).
+* repeated calls on one workspace give the same block lists and pooled keys
+  bit for bit, and outputs equal up to the rounding of the fp32 merge (how a
+  row's blocks are split among CTAs depends on timing, so the order in which
+  partial results are combined does too): within REPEAT_TOL of each other;
+  the gate's row counters reset themselves, the launch counter grows by one
+  grid per call and tags every row the call publishes.
 """
 import numpy as np
 import pytest
@@ -21,6 +24,12 @@ from oracle import oracle as O
 from gpu_helpers import check_attention, check_indices, oracle_bits, to_dev
 
 pytestmark = pytest.mark.gpu
+
+# Two calls on the same inputs may split a row's blocks differently among the
+# CTAs (the decode takes work dynamically), so their bf16 outputs may differ by
+# the rounding of the fp32 merge: at most a bf16 unit in the last place or two.
+REPEAT_TOL = 4e-3
+REPEAT_LSE_TOL = 2e-5
 
 
 def run_both(wl, inp):
@@ -88,29 +97,75 @@ def test_fused_repeated_calls_reuse_workspace():
         torch.cuda.synchronize()
         outs.append((st.out.clone(), st.lse.clone(), st.block_idx.clone()))
     for o, l, i in outs[1:]:
-        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1]) and torch.equal(i, outs[0][2])
+        assert torch.equal(i, outs[0][2])
+        assert (o.float() - outs[0][0].float()).abs().max().item() <= REPEAT_TOL
+        assert (l - outs[0][1]).abs().max().item() <= REPEAT_LSE_TOL
     ws = st.workspace()
-    # the grid barrier's 64-bit arrival counter grows by one grid (one CTA per SM) per call
+    # the 64-bit launch counter grows by one grid (one CTA per SM) per call
     arrivals = int(ws[:8].view(torch.int64).item())
     assert arrivals == 4 * torch.cuda.get_device_properties(0).multi_processor_count
     assert api.seer_decode_wait_failures() == 0
 
 
-def test_fused_one_cta_per_row_needs_no_barrier():
-    # 80 rows on a 148-SM part: one CTA per row in both phases, a plain launch of 80
-    # CTAs; the grid barrier's counter is never touched
+def _state(st, rows):
+    ws = st.workspace()
+    off = (256 + rows * 4 + 255) // 256 * 256  # per-row decode states, 32 bytes each
+    state = ws[off:off + rows * 32].view(torch.int32).view(rows, 8).cpu().numpy()
+    return ws, state  # columns: ready epoch, slots handed out, front, back, positions counted in
+
+
+def _three_calls(wl, inp):
+    st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
+    st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
+    outs = []
+    for _ in range(3):
+        st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+        torch.cuda.synchronize()
+        outs.append(st.out.clone())
+    assert all((o.float() - outs[0].float()).abs().max().item() <= REPEAT_TOL for o in outs[1:])
+    return st
+
+
+def test_fused_launch_epochs_rows_fit_the_grid():
+    # 80 rows on a 148-SM part: each row is gated by one CTA, which then streams
+    # the whole row and writes the output directly. Every call adds one grid (one
+    # CTA per SM) to the launch counter and publishes every row with its epoch, so
+    # nothing is reset between calls.
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     rows = sms // 2 + 6
     wl = W.Workload("rows", rows // 2, 8, 2, 128, 128, 64, 1024, 256)
     lens = np.array([1024 - 7 * b for b in range(wl.batch)], np.int32)
     inp = to_dev(W.make_inputs(wl, seed=21, pad_value=float("nan"), seq_lens=lens))
     check_step(wl, inp)
-    st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
-    st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
-    for _ in range(3):
-        st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
-    torch.cuda.synchronize()
-    assert int(st.workspace()[:8].view(torch.int64).item()) == 0
+    st = _three_calls(wl, inp)
+    ws, state = _state(st, rows)
+    assert int(ws[:8].view(torch.int64).item()) == 3 * sms
+    assert np.all(state[:, 0] == 3)  # published by the third call
+    assert np.all(state[:, 4] == 0)  # one CTA per row: no partial slot was counted
+    assert api.seer_decode_wait_failures() == 0
+
+
+def test_fused_rows_outnumber_the_grid_take_and_help():
+    # More rows than SMs: CTAs take pieces of each row's list from the front and
+    # help with the rows that have most left from the back. After three calls the
+    # tally of fully taken rows (kept by launch parity) counts every row for the
+    # third call and has been cleared for the fourth; every row's front met its back.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, Hkv = (sms + 40) // 4 + 1, 4
+    rows = B * Hkv
+    wl = W.Workload("many", B, 16, Hkv, 128, 128, 64, 2048, 512)
+    lens = np.array([2048 - 37 * (b % 40) for b in range(B)], np.int32)
+    inp = to_dev(W.make_inputs(wl, seed=22, pad_value=float("nan"), seq_lens=lens))
+    check_step(wl, inp, batches=[0, 1, B - 1])
+    st = _three_calls(wl, inp)
+    ws, state = _state(st, rows)
+    assert int(ws[:8].view(torch.int64).item()) == 3 * sms
+    tally = ws[8:16].view(torch.int32).cpu().numpy()  # by launch parity: epoch 3 counts in word 1
+    assert tally[1] == rows and tally[0] == 0
+    nsel = st.num_selected.view(-1).cpu().numpy()
+    assert np.all(state[:, 0] == 3)
+    assert np.all(state[:, 2] >= state[:, 3])                       # front met back: all taken
+    assert np.all((state[:, 4] == nsel) | (state[:, 4] == 0))       # counted in fully, or one whole run
     assert api.seer_decode_wait_failures() == 0
 
 

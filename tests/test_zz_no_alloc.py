@@ -4,10 +4,14 @@ Some callers cannot give the step a device workspace -- a plugin that its
 host framework hands only input and output tensors, or a serving loop that
 may not call cudaMalloc once it runs. This entry point keeps the step's
 scratch in a static device array inside the library instead. Called through
-the C ABI, two calls in a row must each reproduce the output of the
-workspace entry point (seer_decode_step) on the same inputs, within the
-attention tolerance of the parity tests; sizes whose scratch exceeds the
-array are refused with SEER_ERR_UNSUPPORTED.
+the C ABI, two calls in a row must each reproduce the workspace entry point
+(seer_decode_step) on the same inputs: block lists and pooled keys bit for
+bit, outputs within the rounding by which two calls of the same kernel may
+differ (the decode splits rows among CTAs dynamically, so the fp32 merge
+order varies) -- far inside the attention tolerance of the parity tests.
+A second, different shape runs in the same loop on the array the first left
+behind. Sizes whose scratch exceeds the array are refused with
+SEER_ERR_UNSUPPORTED.
 
 This file is collected last on purpose, and passes both alone in a fresh
 process and after every other test (the array keeps the previous call's
@@ -24,7 +28,8 @@ from block_sparse_attention_seer_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-OUT_MAX_ABS = 1e-2  # the attention tolerance of the parity tests
+OUT_MAX_ABS = 4e-3  # a bf16 unit or two in the last place: the merge-order rounding of two calls
+LSE_MAX_ABS = 2e-5
 
 
 def _outputs(wl, kpool0):
@@ -44,31 +49,37 @@ def _call_noalloc(dims, inp, wl, o):
         o["lse"].data_ptr(), torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("name", ["decode_b16", "tiny"])
-def test_noalloc_matches_workspace_entry_two_calls(name):
+def _reference(name):
     wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl, seed=21, device="cuda")
-    dims = api.make_dims(**wl.dims())
     ref_st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens)
     ref_st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
     kpool0 = ref_st.kpool.clone()
     ref_st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
     torch.cuda.synchronize()
+    return wl, inp, api.make_dims(**wl.dims()), ref_st, kpool0
+
+
+@pytest.mark.parametrize("names", [("decode_b16", "tiny"), ("tiny", "decode_b16")])
+def test_noalloc_matches_workspace_entry_two_calls(names):
+    cases = [_reference(n) for n in names]
     for _ in range(2):
-        o = _outputs(wl, kpool0)
-        assert _call_noalloc(dims, inp, wl, o) == api.SEER_OK, api.LIB.seer_last_error_string().decode()
-        torch.cuda.synchronize()
-        err = (o["out"].float() - ref_st.out.float()).abs().max().item()
-        assert err <= OUT_MAX_ABS, err
-        assert torch.isfinite(o["out"].float()).all()
-        np.testing.assert_allclose(o["lse"].cpu().numpy(), ref_st.lse.cpu().numpy(), rtol=0, atol=1e-3)
-        assert torch.equal(o["block_idx"], ref_st.block_idx)
-        assert torch.equal(o["num_selected"], ref_st.num_selected)
-        assert torch.equal(o["kpool"], ref_st.kpool)
+        for wl, inp, dims, ref_st, kpool0 in cases:  # each shape on the array the other left
+            o = _outputs(wl, kpool0)
+            assert _call_noalloc(dims, inp, wl, o) == api.SEER_OK, api.LIB.seer_last_error_string().decode()
+            torch.cuda.synchronize()
+            assert torch.isfinite(o["out"].float()).all()
+            err = (o["out"].float() - ref_st.out.float()).abs().max().item()
+            assert err <= OUT_MAX_ABS, err
+            np.testing.assert_allclose(o["lse"].cpu().numpy(), ref_st.lse.cpu().numpy(), rtol=0, atol=LSE_MAX_ABS)
+            assert torch.equal(o["block_idx"], ref_st.block_idx)
+            assert torch.equal(o["num_selected"], ref_st.num_selected)
+            assert torch.equal(o["kpool"], ref_st.kpool)
 
 
 def test_noalloc_refuses_sizes_beyond_the_static_array():
-    wl = W.WORKLOADS["ragged"]  # 64 sequences x 32 heads of split partials: well above 32 MiB
+    # 128 sequences x 32 heads of partial slots: above 32 MiB
+    wl = W.WORKLOADS["ragged"].with_(batch=128)
     dims = api.make_dims(**wl.dims())
     assert api.seer_decode_step_workspace_size(dims, wl.budget_tokens) > (32 << 20)
     fake = torch.empty(256, dtype=torch.uint8, device="cuda")  # never read: refused before any launch
