@@ -1033,7 +1033,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
 
     // Stream one run of `row` (nsel list positions) from the piece [a0, a1) it holds;
     // from the front, further pieces are claimed one ahead until the row has none left.
-    auto run = [&](int row, int nsel, int a0, int a1, bool from_front, const int* head) {
+    auto run = [&](int row, int nsel, int a0, int a1, bool from_front, const int* head, int fixed_slot) {
         const int b = row / p.Hkv;
         const int L = clamp_len(p.seq_lens[b], p.Lmax);
         const int NB = (L + BLK - 1) / BLK;
@@ -1043,6 +1043,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
         int n1 = chunk;
         if (lane == 0) {
             slot = atomicAdd(&f.rs[row].nslots, 1u);  // needed at the run's end
+            if (fixed_slot >= 0) slot = (unsigned int)fixed_slot;
             if (from_front) {
                 n1 = max(chunk, (nsel - a1) / 8);  // an eighth of what may be left, at least a chunk
                 c1 = atomicAdd(&f.rs[row].span, (unsigned long long)n1);
@@ -1122,7 +1123,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
         a0 = __shfl_sync(kFull, a0, 0);
         a1 = __shfl_sync(kFull, a1, 0);
         nsel = __shfl_sync(kFull, nsel, 0);
-        if (a0 < a1) run(row, nsel, a0, a1, true, nullptr);
+        if (a0 < a1) run(row, nsel, a0, a1, true, nullptr, -1);
     };
 
     const int nselrows = sel.count;
@@ -1148,7 +1149,10 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
             if (ok) {
                 const int a0 = (int)((long long)part * nsel / f.gate_cpr);
                 const int a1 = (int)((long long)(part + 1) * nsel / f.gate_cpr);
-                if (a0 < a1) run(row, nsel, a0, a1, false, a0 == 0 ? head : nullptr);
+                // a fixed slot per non-empty part: the merge adds the parts in the same
+                // order on every call, so the output is the same bit for bit
+                const int slot = nsel >= f.gate_cpr ? part : a0;
+                if (a0 < a1) run(row, nsel, a0, a1, false, a0 == 0 ? head : nullptr, slot);
             }
         }
         if (ok) put(0, 0, 0, kExit, 0, 0, 0, false);
@@ -1163,7 +1167,8 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
 
     // ---- rows outnumber the CTAs:
     // ---- 1. the rows this CTA selected, from the chunk it kept
-    for (int i = 0; ok && i < nselrows; ++i) run(sel.row[i], sel.nsel[i], 0, min(chunk, sel.nsel[i]), true, sel.head[i]);
+    for (int i = 0; ok && i < nselrows; ++i)
+        run(sel.row[i], sel.nsel[i], 0, min(chunk, sel.nsel[i]), true, sel.head[i], -1);
 
     // ---- 2. its other home rows
     int home_lo, home_hi;
@@ -1221,7 +1226,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
             a0 = __shfl_sync(kFull, a0, 0);
             a1 = __shfl_sync(kFull, a1, 0);
             nsel = __shfl_sync(kFull, nsel, 0);
-            if (a0 < a1) run(row, nsel, a0, a1, false, nullptr);
+            if (a0 < a1) run(row, nsel, a0, a1, false, nullptr, -1);
             empty_windows = 0;
             idle_since = 0;
             continue;  // look at the same window again
@@ -1586,11 +1591,14 @@ StepGeometry step_geometry(const Shape& s, int kmax, int num_sms) {
     }
     // about 64 KB of K+V per claim, at most 64 claims per row. A run holds at
     // least one whole chunk except the front and the back piece that meet, so
-    // a row has at most chunks + 2 runs, each with its slot.
+    // a row has at most chunks + 2 runs, each with its slot; with fixed parts
+    // (rows fit the grid) a row has min(kmax, CTAs per row) non-empty parts.
     const int base = s.blk == 64 ? 2 : 1;
     const int c = (kmax + 63) / 64;
     g.chunk = c < base ? base : c;
     g.nslots = (kmax + g.chunk - 1) / g.chunk + 2;
+    const int parts = kmax < g.gate_cpr ? kmax : g.gate_cpr;
+    if (parts > g.nslots) g.nslots = parts;
     return g;
 }
 

@@ -118,3 +118,77 @@ def test_prefill_matches_oracle(shape):
 @pytest.mark.parametrize("blk", [64, 128])
 def test_prefill_dense_lists(blk):
     check(make(2, 4, 2, 128, 128, blk, 512, [512, 333], seed=blk), budget=blk, dense=True)
+
+
+def attend_lists(c, lists, kmax):
+    """The prefill attention on given per-query-block lists, against the oracle on the same lists."""
+    B, Hq, Lmax, D = c["q"].shape
+    Hkv = c["k"].shape[1]
+    blk = c["blk"]
+    nbm = -(-Lmax // blk)
+    idx = np.full((B, Hkv, nbm, kmax), -1, np.int32)
+    ns = np.zeros((B, Hkv, nbm), np.int32)
+    for i, lst in enumerate(lists):
+        idx[:, :, i, :len(lst)] = lst
+        ns[:, :, i] = len(lst)
+    dims = api.make_dims(B, Hq, Hkv, D, 128, blk, Lmax)
+    out = torch.empty(B, Hq, Lmax, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Hq, Lmax, device="cuda")
+    lens = torch.from_numpy(c["lens"]).cuda()
+    api.seer_prefill_attention(dims, c["q"].cuda(), c["k"].cuda(), c["v"].cuda(), lens, torch.from_numpy(idx).cuda(),
+                               torch.from_numpy(ns).cuda(), kmax, out, lse)
+    torch.cuda.synchronize()
+    o_out, o_lse = O.prefill_attend(u16(c["q"]), u16(c["k"]), u16(c["v"]), c["lens"], idx, ns, blk)
+    g_out, g_lse = out.cpu().double().numpy(), lse.cpu().double().numpy()
+    L = int(c["lens"][0])
+    d = np.abs(g_out[0, :, :L] - o_out[0, :, :L])
+    # the output is bf16: a token that sees one or two keys returns a V row of magnitude up to
+    # ~5, where half a bf16 unit in the last place is 2^-6; the bound adds that rounding
+    bound = 1e-2 + 2.0 ** -7 * np.abs(o_out[0, :, :L])
+    assert np.all(d <= bound), (d.max(), (d - bound).max())
+    assert d.mean() <= 1e-3, d.mean()
+    assert np.abs(g_lse[0, :, :L] - o_lse[0, :, :L]).max() <= 1e-3
+    return g_out, o_out
+
+
+def late_lists(nb, late, keep, rng):
+    """Each query block keeps only itself, except the last `late`, which keep `keep` blocks:
+    themselves and keep - 1 earlier ones drawn at random (ascending lists)."""
+    lists = []
+    for i in range(nb):
+        if i < nb - late:
+            lists.append([i])
+        else:
+            lists.append(sorted(rng.choice(i, size=keep - 1, replace=False).tolist()) + [i])
+    return lists
+
+
+def test_prefill_deep_lists_wrap_the_rings():
+    # an 8K-token prompt; the last three query blocks keep 64 blocks (a 4K-token budget):
+    # 32 key sub-tiles per query tile, so the 2-slot K ring and the 3-slot V ring wrap
+    # 16 and 10 times
+    c = make(1, 4, 1, 128, 128, 64, 8192, [8192], seed=81)
+    rng = np.random.default_rng(81)
+    attend_lists(c, late_lists(128, 3, 64, rng), 64)
+
+
+def test_prefill_late_salient_block_rescales():
+    # the last three query blocks keep 64 blocks; in each list, the last earlier block
+    # has its keys scaled x8 (exact in bf16), so a row's maximum grows by far more than
+    # 2^8 after the first sub-tiles and the running output and sum are rescaled
+    c = make(1, 4, 1, 128, 128, 64, 8192, [8192], seed=82)
+    rng = np.random.default_rng(82)
+    lists = late_lists(128, 3, 64, rng)
+    for lst in lists[-3:]:
+        j = lst[-2]
+        c["k"][:, :, j * 64:(j + 1) * 64] = (c["k"][:, :, j * 64:(j + 1) * 64].float() * 8).to(torch.bfloat16)
+    g_out, _ = attend_lists(c, lists, 64)
+    assert np.isfinite(g_out[0, :, -192:]).all()
+
+
+def test_prefill_lists_longer_than_the_staged_limit():
+    # 400 blocks of 64: the last two query blocks keep every block (399 and 400 entries, more
+    # than the 384 list entries a CTA stages in shared memory), read from global memory
+    c = make(1, 4, 1, 128, 128, 64, 64 * 400, [64 * 400], seed=83)
+    lists = [[i] for i in range(398)] + [list(range(399)), list(range(400))]
+    attend_lists(c, lists, 400)
