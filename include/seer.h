@@ -306,14 +306,23 @@ seer_status seer_append_kv(const seer_dims* dims, const void* k_new, const void*
                            void* k_cache, void* v_cache, cudaStream_t stream);
 
 /*
- * The whole decode step, a1..a5, in ONE cooperative launch (one CTA per SM).
- * Phase 1 spreads the (b, kvh) rows over the CTAs: refresh kpool for the
- * blocks touching [upd_start[b], L_b) (NULL: the last block only, i.e. the
- * token just appended), score every other block with the same arithmetic
- * as seer_gate_scores, and select as seer_select_blocks does (bit-identical
- * block lists). After a grid-wide barrier, phase 2 is seer_sparse_decode's
- * schedule; the last CTA to finish a row merges its slots into out / lse_out
- * as seer_combine does. One launch, no host synchronisation.
+ * The whole decode step, a1..a5, in ONE cooperative launch (one CTA per SM),
+ * with no grid-wide barrier. The gate spreads the pooled-key positions of the
+ * (b, kvh) rows over the CTAs: it refreshes kpool for the blocks touching
+ * [upd_start[b], L_b) (NULL: the last block only, i.e. the token just
+ * appended), scores every other block with the same arithmetic as
+ * seer_gate_scores and selects as seer_select_blocks does (bit-identical
+ * block lists); the CTA that completes a row's gate publishes the row (a
+ * release flag). The decode of a row starts as soon as it is published: when
+ * rows fit the grid, the CTAs that gated a row stream even, fixed parts of its
+ * kept list (a row held by one CTA is written straight to out); when rows
+ * outnumber the CTAs, CTAs take pieces of each list from the front and help
+ * with the rows that have most left from the back. The CTA that completes a
+ * row's positions merges its partial results into out / lse_out as
+ * seer_combine does. One launch, no host synchronisation.
+ * (The step of "SeerAttention-R: Sparse Attention Adaptation for Long
+ * Reasoning", abstract; gate of "SeerAttention: Learning Intrinsic Sparse
+ * Attention in Your LLMs", abstract.)
  *
  *   q, k_cache, v_cache, w_q, w_k, seq_lens   as above
  *   upd_start     int32 [B] or NULL (NULL: L_b - 1)
@@ -325,10 +334,19 @@ seer_status seer_append_kv(const seer_dims* dims, const void* k_new, const void*
  *   out           bf16 [B, Hq, D]      (output)
  *   lse_out       fp32 [B, Hq]         (output, may be NULL)
  *   workspace     device scratch of at least seer_decode_step_workspace_size()
- *                 bytes, 256-byte aligned, ZERO-FILLED before its first use; every
- *                 call leaves it ready for the next one (re-zero it after a call
- *                 that reported a wait failure). Calls that share a workspace
- *                 must not overlap on the GPU.
+ *                 bytes, 256-byte aligned, ZERO-FILLED before its first use on a
+ *                 device; every call leaves it ready for the next one (each
+ *                 launch takes the next epoch from a counter in it and tags
+ *                 what it publishes with that epoch; re-zero it after a call
+ *                 that reported a wait failure). Use one workspace with one
+ *                 device only. Calls that share a workspace must not overlap
+ *                 on the GPU.
+ * Repeatability: block_idx, num_selected and kpool are the same bit for bit on
+ * every call with the same inputs. With no more (b, kvh) rows than SMs, out and
+ * lse_out are too (fixed parts merged in a fixed order); with more rows, the
+ * split of a row among CTAs depends on timing and out / lse_out may differ
+ * between calls by the rounding of the fp32 merge (a bf16 unit in the last
+ * place at most, in practice).
  * Errors: as the separate calls; SEER_ERR_CUDA also when the cooperative launch
  * cannot place one CTA on every SM (e.g. the device is shared with other work).
  */
