@@ -142,6 +142,7 @@ struct Smem {
     __device__ __forceinline__ uint32_t cons() const { return bars + 16u * nst; }
     __device__ __forceinline__ uint32_t gate(int st) const { return bars + 16u * nst + 8u + 8u * st; }
     __device__ __forceinline__ uint32_t helper() const { return bars + 16u * nst + 8u + 8u * kMaxGateStages; }
+    __device__ __forceinline__ uint32_t wq() const { return bars + 16u * nst + 16u + 8u * kMaxGateStages; }
 };
 
 __device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) {
@@ -161,6 +162,7 @@ __device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) 
         mbar_init(m.cons(), kConsumerWarps);  // one arrival per warp (warp_group_sync)
         for (int st = 0; st < kMaxGateStages; ++st) mbar_init(m.gate(st), 1);
         mbar_init(m.helper(), kHelperThreads / 32);
+        mbar_init(m.wq(), 1);
         for (int i = 0; i < kInfoWords; ++i) m.info[i] = 0;
         fence_mbar_init();
     }
@@ -614,6 +616,7 @@ struct StepParams {
     int gate_cpr;                            // CTAs per row when rows fit the grid, else 0
     int chunk;                               // list positions per claim from the front
     int keys_off, chunk_off, n_gate_stages;  // gate keys and pooled-key copies inside the stage ring
+    int wq_stages;                           // rows fit the grid: the last gate stages first hold W_q
     int sel_off;                             // rows this CTA selected (shared memory, kMaxSelRows)
     int refresh_off;                         // pool scratch of the helper warps (outside the ring)
 };
@@ -651,6 +654,14 @@ __device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) 
 // the word of its epoch's parity, which the previous launch cleared, and
 // clears the other word for the next launch (launches on one workspace run in
 // stream order). Counting is a fire-and-forget add: no thread waits on it.
+// The launch's epoch from the launch counter's old value. The empty asm keeps
+// the division (and so the wait for the counter's atomic) at the point of use:
+// the atomic is issued at kernel entry and returns while the gate's loads run.
+__device__ __forceinline__ uint32_t epoch_of(unsigned long long old_ctr) {
+    asm volatile("" : "+l"(old_ctr));
+    return (uint32_t)(old_ctr / gridDim.x) + 1u;  // every launch adds gridDim.x
+}
+
 __device__ __forceinline__ void count_taken_row(unsigned int* tally, uint32_t epoch) {
     atomicAdd(tally + (epoch & 1u), 1u);
 }
@@ -672,8 +683,11 @@ constexpr int kMaxBatchRows = 8;
 constexpr int kMaxSelRows = 32;
 struct SelList {
     int count;
+    int publish;  // rows fit the grid: the row this CTA selected, released after the gate (else -1)
+    int own_len;  // rows fit the grid: the length of the row this CTA gated
     int row[kMaxSelRows];
     int nsel[kMaxSelRows];
+    int len[kMaxSelRows];
     int head[kMaxSelRows][kSelectHead];  // the first list entries of each
 };
 
@@ -700,9 +714,10 @@ static_assert(sizeof(GateScratch<64, 128>) <= kGateScratchBytes, "gate scratch")
 // select its blocks and publish the row. The open last block is never a
 // candidate, so its pooled key is refreshed by the helper warps during the
 // decode; only blocks that compete (a refresh point before the last block)
-// are refreshed here. `epoch` is valid in thread 0.
+// are refreshed here. `old_ctr` (the launch counter before this CTA's add) is
+// valid in thread 0.
 template <int D, int BLK, int DG>
-__device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, uint32_t epoch) {
+__device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, unsigned long long old_ctr) {
     constexpr int kThreads = kStepThreads;
     constexpr int kWarps = kThreads / 32;
     constexpr int kChunkRows = kGateChunkBytes / (DG * 4);
@@ -724,6 +739,19 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
     // range strictly inside a row still counts for that row).
     const int r_stop = (int)((h1 + f.NBmax - 1) / f.NBmax);
     int chunk_it = 0;  // bulk copies consumed so far (the same count on every thread)
+    // Rows fit the grid (one row per CTA): W_q of the row's head arrives by one
+    // bulk copy into the last wq_stages gate stages, so no register loads sit
+    // in front of the length load and the first pooled-key copies; those
+    // stages join the ring once the projection has read them.
+    const int wq_stages = f.wq_stages;
+    const int n_first = f.n_gate_stages - wq_stages;  // gate stages free before the projection
+    const float* wq_s = reinterpret_cast<const float*>(m.base + f.chunk_off + n_first * kGateChunkBytes);
+    if (wq_stages > 0 && tid == 0) {
+        const uint32_t bytes = (uint32_t)(DG * D * 4);
+        mbar_arrive_expect_tx(m.wq(), bytes);
+        bulk_load(m.sbase + (uint32_t)(f.chunk_off + n_first * kGateChunkBytes),
+                  f.w_q + (size_t)((int)(h0 / f.NBmax) % p.Hkv) * DG * D, bytes, m.wq());
+    }
 
     for (int r = (int)(h0 / f.NBmax); r < r_stop;) {
         const int nb = min(kMaxBatchRows, r_stop - r);
@@ -741,7 +769,7 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
             if (f.upd_start) upd_raw = load_early(f.upd_start + b);
         }
         WVec w[kQBatch];
-        if (total_q > 0) {
+        if (total_q > 0 && wq_stages == 0) {
 #pragma unroll
             for (int u = 0; u < kQBatch; ++u) {
                 const int o = min(warp + u * kWarps, total_q - 1);
@@ -760,17 +788,6 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
             g.NB = (g.L + BLK - 1) / BLK;
             const int st0 = max(f.upd_start ? upd_raw : g.L - 1, 0);  // as refresh_start_block
             g.js = g.NB > 0 ? min(st0 / BLK, g.NB) : g.NB;
-        }
-        if (total_q > 0) {
-            for (int idx = tid; idx < nb * D; idx += kThreads) {
-                const int k = idx / D, d = idx - k * D;
-                const int row = r + k, b = row / p.Hkv, kvh = row - b * p.Hkv;
-                sm.qbar[k][d] = group_query_mean_at(p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G) * D, p.G, D, d);
-            }
-        }
-        __syncthreads();
-        if (tid < nb) {
-            GateRow& g = sm.rows[tid];
             const long long rs = (long long)g.r * f.NBmax;
             const int i0 = (int)(h0 > rs ? h0 - rs : 0);
             const int i1 = (int)((h1 - rs) < f.NBmax ? (h1 - rs) : f.NBmax);
@@ -781,11 +798,14 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
             g.s0 = min(i0, lim);
             g.s1 = min(i1, lim);
             g.refresh_now = g.js < ncand && g.js >= i0 && g.js < i1;
+            if (f.gate_cpr > 0) reinterpret_cast<SelList*>(m.base + f.sel_off)->own_len = g.L;  // nb == 1
         }
-        __syncthreads();
         auto nchunks_of = [&](int k) { return (sm.rows[k].s1 - sm.rows[k].s0 + kChunkRows - 1) / kChunkRows; };
-        int total_chunks = 0;
-        for (int k = 0; k < nb; ++k) total_chunks += nchunks_of(k);
+        auto count_chunks = [&]() {
+            int n = 0;
+            for (int k = 0; k < nb; ++k) n += nchunks_of(k);
+            return n;
+        };
         auto chunk = [&](int i, int& k, int& j0, int& n) {
             for (k = 0; k < nb - 1; ++k) {
                 const int c = nchunks_of(k);
@@ -804,10 +824,47 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
             bulk_load(m.sbase + (uint32_t)(f.chunk_off + stage * kGateChunkBytes),
                       f.kpool + ((size_t)sm.rows[k].r * f.NBmax + j0) * DG, bytes, m.gate(stage));
         };
-        // ---- (2) stream the cached pooled keys; meanwhile project the batch rows' queries
-        if (tid == 0)
-            for (int i = 0; i < min(f.n_gate_stages, total_chunks); ++i) issue(i);
+        // ---- (2) stream the cached pooled keys; meanwhile project the batch rows' queries.
+        //      One row per CTA: thread 0 wrote the row itself and issues its first
+        //      copies before the group-mean query.
+        if (tid == 0 && wq_stages > 0) {  // nb == 1: the row thread 0 just wrote
+            const int n0 = count_chunks();
+            for (int i = 0; i < min(n_first, n0); ++i) issue(i);
+        }
         if (total_q > 0) {
+            // one row per CTA: warp 0 stays free for the length and the copies
+            const int q0 = wq_stages > 0 ? 32 : 0;
+            for (int idx = tid - q0; idx >= 0 && idx < nb * D; idx += kThreads - q0) {
+                const int k = idx / D, d = idx - k * D;
+                const int row = r + k, b = row / p.Hkv, kvh = row - b * p.Hkv;
+                sm.qbar[k][d] = group_query_mean_at(p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G) * D, p.G, D, d);
+            }
+        }
+        __syncthreads();
+        const int total_chunks = count_chunks();
+        if (tid == 0 && wq_stages == 0)
+            for (int i = 0; i < min(f.n_gate_stages, total_chunks); ++i) issue(i);
+        if (wq_stages > 0) {
+            // the same pieces and sums as the register path below (equal bits)
+            constexpr int kPerWarp = (DG + kWarps - 1) / kWarps;
+            if (!mbar_wait(m.wq(), 0u)) record_failure(m.info);
+#pragma unroll 1
+            for (int u0 = 0; u0 < kPerWarp; u0 += 4) {  // four outputs per warp in flight
+                WVec wv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = min(warp + (u0 + u) * kWarps, DG - 1);
+                    wv[u] = *reinterpret_cast<const WVec*>(wq_s + (size_t)e * D + lane * kVecD);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = warp + (u0 + u) * kWarps;
+                    const float x = warp_sum(piece_dot(wv[u], &sm.qbar[0][lane * kVecD]));
+                    if (lane == 0 && e < DG) sm.qg[0][e] = x;
+                }
+            }
+            fence_proxy_async_smem();  // these generic reads of W_q precede the copies into its stages
+        } else if (total_q > 0) {
 #pragma unroll
             for (int u = 0; u < kQBatch; ++u) {
                 const int o = warp + u * kWarps;
@@ -835,6 +892,8 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
             }
         }
         __syncthreads();
+        if (tid == 0 && wq_stages > 0)  // the W_q stages are read: they join the ring
+            for (int i = n_first; i < min(f.n_gate_stages, total_chunks); ++i) issue(i);
 
         // ---- (3) refresh and score competing blocks of a refresh point inside the range (multi-token appends)
         for (int k = 0; k < nb; ++k) {
@@ -924,6 +983,7 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
                 if (keep) {
                     sel.row[sel.count] = g.r;
                     sel.nsel[sel.count] = kb;
+                    sel.len[sel.count] = g.L;
                     ++sel.count;
                 }
             }
@@ -937,8 +997,13 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
             }
             __syncthreads();  // the list, the count and the state before the release
             if (tid == 0) {
-                if (f.gate_cpr == 0 && kept == kb) count_taken_row(f.rows_taken, epoch);  // nothing left to take
-                st_release_u32(&f.rs[g.r].ready, epoch);
+                if (f.gate_cpr > 0) {
+                    sel.publish = g.r;  // released after the gate, so the producer starts first
+                } else {
+                    const uint32_t epoch = epoch_of(old_ctr);
+                    if (kept == kb) count_taken_row(f.rows_taken, epoch);  // nothing left to take
+                    st_release_u32(&f.rs[g.r].ready, epoch);
+                }
             }
         }
         fence_proxy_async_smem();
@@ -1033,17 +1098,16 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
 
     // Stream one run of `row` (nsel list positions) from the piece [a0, a1) it holds;
     // from the front, further pieces are claimed one ahead until the row has none left.
-    auto run = [&](int row, int nsel, int a0, int a1, bool from_front, const int* head, int fixed_slot) {
+    auto run = [&](int row, int nsel, int a0, int a1, bool from_front, const int* head, int fixed_slot, int Lrow) {
         const int b = row / p.Hkv;
-        const int L = clamp_len(p.seq_lens[b], p.Lmax);
+        const int L = Lrow >= 0 ? Lrow : clamp_len(p.seq_lens[b], p.Lmax);
         const int NB = (L + BLK - 1) / BLK;
         const int32_t* list = f.block_idx + (size_t)row * p.kmax;
         unsigned int slot = 0;
         unsigned long long c1 = 0;  // lane 0: the claim in flight, of n1 positions
         int n1 = chunk;
         if (lane == 0) {
-            slot = atomicAdd(&f.rs[row].nslots, 1u);  // needed at the run's end
-            if (fixed_slot >= 0) slot = (unsigned int)fixed_slot;
+            slot = fixed_slot >= 0 ? (unsigned int)fixed_slot : atomicAdd(&f.rs[row].nslots, 1u);  // needed at the run's end
             if (from_front) {
                 n1 = max(chunk, (nsel - a1) / 8);  // an eighth of what may be left, at least a chunk
                 c1 = atomicAdd(&f.rs[row].span, (unsigned long long)n1);
@@ -1123,7 +1187,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
         a0 = __shfl_sync(kFull, a0, 0);
         a1 = __shfl_sync(kFull, a1, 0);
         nsel = __shfl_sync(kFull, nsel, 0);
-        if (a0 < a1) run(row, nsel, a0, a1, true, nullptr, -1);
+        if (a0 < a1) run(row, nsel, a0, a1, true, nullptr, -1, -1);
     };
 
     const int nselrows = sel.count;
@@ -1152,7 +1216,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
                 // a fixed slot per non-empty part: the merge adds the parts in the same
                 // order on every call, so the output is the same bit for bit
                 const int slot = nsel >= f.gate_cpr ? part : a0;
-                if (a0 < a1) run(row, nsel, a0, a1, false, a0 == 0 ? head : nullptr, slot);
+                if (a0 < a1) run(row, nsel, a0, a1, false, a0 == 0 ? head : nullptr, slot, sel.own_len);
             }
         }
         if (ok) put(0, 0, 0, kExit, 0, 0, 0, false);
@@ -1168,7 +1232,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
     // ---- rows outnumber the CTAs:
     // ---- 1. the rows this CTA selected, from the chunk it kept
     for (int i = 0; ok && i < nselrows; ++i)
-        run(sel.row[i], sel.nsel[i], 0, min(chunk, sel.nsel[i]), true, sel.head[i], -1);
+        run(sel.row[i], sel.nsel[i], 0, min(chunk, sel.nsel[i]), true, sel.head[i], -1, sel.len[i]);
 
     // ---- 2. its other home rows
     int home_lo, home_hi;
@@ -1226,7 +1290,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
             a0 = __shfl_sync(kFull, a0, 0);
             a1 = __shfl_sync(kFull, a1, 0);
             nsel = __shfl_sync(kFull, nsel, 0);
-            if (a0 < a1) run(row, nsel, a0, a1, false, nullptr, -1);
+            if (a0 < a1) run(row, nsel, a0, a1, false, nullptr, -1, -1);
             empty_windows = 0;
             idle_since = 0;
             continue;  // look at the same window again
@@ -1299,8 +1363,11 @@ __device__ __forceinline__ bool step_flush(const Params& p, const StepParams& f,
     if (whole) return true;
     if (ctid == 0) {
         const unsigned int before = atomic_add_acq_rel(&f.rs[row].done, (unsigned int)nrun);
-        // every run of the row took its slot before it counted: the last count sees them all
-        const int ns = (before + (unsigned int)nrun == (unsigned int)nsel) ? (int)ld_relaxed_u32(&f.rs[row].nslots) : 0;
+        // every run of the row took its slot before it counted: the last count sees them all;
+        // fixed parts (rows fit the grid) fill slots 0 .. min(nsel, parts) - 1
+        const int ns = (before + (unsigned int)nrun != (unsigned int)nsel) ? 0
+                       : f.gate_cpr > 0                                    ? min(nsel, f.gate_cpr)
+                                                                           : (int)ld_relaxed_u32(&f.rs[row].nslots);
         *reinterpret_cast<volatile int*>(m.info + kInfoMergeRow) = min(ns, p.S);
     }
     __syncwarp();
@@ -1449,26 +1516,38 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                        const Params p, const StepParams f) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const Smem m = setup_smem(smem_raw, p);
-    uint32_t epoch = 0;
+    unsigned long long old_ctr = 0;
     if (threadIdx.x == 0) {
         prefetch_tensor_map(&tmK);
         prefetch_tensor_map(&tmV);
-        unsigned long long old;
-        asm volatile("atom.add.relaxed.gpu.u64 %0, [%1], 1;" : "=l"(old) : "l"(f.launch_ctr) : "memory");
-        epoch = (uint32_t)(old / gridDim.x) + 1u;  // every launch adds gridDim.x
+        asm volatile("atom.add.relaxed.gpu.u64 %0, [%1], 1;" : "=l"(old_ctr) : "l"(f.launch_ctr) : "memory");
     }
-    if (threadIdx.x == 0) reinterpret_cast<SelList*>(m.base + f.sel_off)->count = 0;  // read after the gate's barriers
-    gate_phase<D, BLK, DG>(p, f, m, epoch);
+    if (threadIdx.x == 0) {  // read after the gate's barriers
+        SelList& sel = *reinterpret_cast<SelList*>(m.base + f.sel_off);
+        sel.count = 0;
+        sel.publish = -1;
+    }
+    gate_phase<D, BLK, DG>(p, f, m, old_ctr);
     fence_proxy_async_smem();  // the gate's use of the ring precedes the decode's copies into it
     if (threadIdx.x == 0) {
+        const uint32_t epoch = epoch_of(old_ctr);
         m.info[kInfoEpoch] = (int)epoch;
         if (blockIdx.x == 0) f.rows_taken[(epoch + 1u) & 1u] = 0u;  // the next launch's tally
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5;
-    if (warp == kConsumerWarps) step_producer<D, BLK>(&tmK, &tmV, p, f, m);
-    else if (warp >= kHelperWarp0) step_helpers<D, BLK>(p, f, m);
-    else step_consumers<D, BLK>(p, f, m);
+    if (warp == kConsumerWarps) {
+        step_producer<D, BLK>(&tmK, &tmV, p, f, m);
+    } else if (warp >= kHelperWarp0) {
+        if (threadIdx.x == kHelperWarp0 * 32) {  // the row this CTA selected (rows fit the grid), after the barrier
+            const int row = reinterpret_cast<const SelList*>(m.base + f.sel_off)->publish;
+            if (row >= 0) st_release_u32(&f.rs[row].ready, (uint32_t)m.info[kInfoEpoch]);
+        }
+        __syncwarp();
+        step_helpers<D, BLK>(p, f, m);
+    } else {
+        step_consumers<D, BLK>(p, f, m);
+    }
 }
 
 // One CTA waits, with the given limit, on an mbarrier that nothing ever
@@ -1501,7 +1580,7 @@ Layout make_layout(int G, bool with_refresh) {
     const int merge_bytes = max(kConsumerWarps * G * D * 4 + 2 * kConsumerWarps * G * 4,  // warp states
                                 with_refresh ? kGateScratchBytes : 0);                   // or the gate's scratch
     const int info_bytes = (kInfoWords + kMaxStages * kStageInfoWords) * 4;
-    const int bar_bytes = (2 * kMaxStages + 2 + kMaxGateStages) * 8;
+    const int bar_bytes = (2 * kMaxStages + 3 + kMaxGateStages) * 8;
     const int refresh_bytes = with_refresh ? (int)sizeof(PoolSmem<D>) + 16 : 0;
     const int sel_bytes = with_refresh ? (int)sizeof(SelList) : 0;
     const int tail = merge_bytes + info_bytes + bar_bytes + refresh_bytes + sel_bytes + 64;
@@ -1657,6 +1736,9 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     f.keys_off = 0;
     f.chunk_off = keys_bytes;
     f.n_gate_stages = n_gate > kMaxGateStages ? kMaxGateStages : n_gate;
+    // rows fit the grid: W_q of the row's head (dg x D fp32) first fills the last gate stages
+    const int wq_st = (DG * D * 4 + kGateChunkBytes - 1) / kGateChunkBytes;
+    f.wq_stages = (geo.gate_cpr > 0 && f.n_gate_stages > wq_st) ? wq_st : 0;
 
     // One CTA per SM, all co-resident (the decode phase waits on rows that other CTAs publish).
     cudaLaunchConfig_t cfg = {};

@@ -276,7 +276,7 @@ def test_workspace_regions_are_disjoint_aligned_and_hold_every_index():
 
 def struct_sizes(D, G):
     pool = (POOL_THREADS // (D // 8)) * D * 4 + D * 4
-    sel_list = 4 + 4 * MAX_SEL_ROWS * 2 + 4 * MAX_SEL_ROWS * SELECT_HEAD
+    sel_list = 4 * 3 + 4 * MAX_SEL_ROWS * 3 + 4 * MAX_SEL_ROWS * SELECT_HEAD  # count, publish, own_len; row, nsel, len; head
     return pool, sel_list
 
 
@@ -285,7 +285,7 @@ def make_layout(D, blk, G, with_refresh):
     stage = (2 * tile + G * D * 2 + 1023) // 1024 * 1024
     merge = max(CONSUMER_WARPS * G * D * 4 + 2 * CONSUMER_WARPS * G * 4, GATE_SCRATCH if with_refresh else 0)
     info = (INFO_WORDS + MAX_STAGES * STAGE_INFO_WORDS) * 4
-    bars = (2 * MAX_STAGES + 2 + MAX_GATE_STAGES) * 8
+    bars = (2 * MAX_STAGES + 3 + MAX_GATE_STAGES) * 8  # full/empty, consumers, gate stages, helpers, W_q
     pool, sel_list = struct_sizes(D, G)
     refresh = pool + 16 if with_refresh else 0
     sel = sel_list if with_refresh else 0
@@ -325,7 +325,17 @@ def test_shared_memory_layout_fits(D, blk, G):
                 keys = (NBmax * 4 + 1023) // 1024 * 1024
                 n_gate = (ring - keys) // GATE_CHUNK
                 assert n_gate >= 1  # at least one pooled-key copy in flight
-                assert keys + min(n_gate, MAX_GATE_STAGES) * GATE_CHUNK <= ring
+                n_gate = min(n_gate, MAX_GATE_STAGES)
+                assert keys + n_gate * GATE_CHUNK <= ring
+                for dg in (64, 128):
+                    # rows that fit the grid: W_q (dg x D fp32, one bulk copy) first fills the
+                    # last wq gate stages, used only when at least one stage stays free for keys
+                    wq_bytes = dg * D * 4
+                    wq = -(-wq_bytes // GATE_CHUNK)
+                    assert wq_bytes % 16 == 0 and wq_bytes < (1 << 20)  # bulk size, mbarrier tx count
+                    if n_gate > wq:
+                        start = keys + (n_gate - wq) * GATE_CHUNK
+                        assert start % 16 == 0 and start + wq_bytes <= keys + n_gate * GATE_CHUNK
 
 
 # ---------------------------------------------------------------- select_row, thread by thread
