@@ -4,10 +4,17 @@
 A step is the whole hot path on one batch: kpool refresh of the open block,
 gate scores, block selection, split-KV sparse decode and the merge of the
 split partials -- run as ONE cooperative launch (seer_decode_step). Inputs are
-seeded synthetic tensors resident in HBM before timing starts. Before every
-timed step a 256 MiB memset flushes L2 and a short device sleep lets the host
-enqueue the step ahead of the GPU; neither is inside the timed interval, a
-pair of CUDA events on the launching stream around the step's launch.
+seeded synthetic tensors resident in HBM before timing starts. Consecutive
+steps rotate over several independent input sets (caches, queries, weights,
+pooled keys; the same lengths), so each step reads inputs that five other
+steps' traffic -- more than the 126 MB L2, in normal-priority data alone --
+has passed through since their last use: cold data, as for one layer of a
+model whose other layers run in between, while the kernel's code stays
+resident as it would in that loop. (--l2 flush instead writes a 256 MiB
+buffer before each step on a single set, which also evicts the code; that
+figure is reported as a secondary key.) A short device sleep before each step
+lets the host enqueue it ahead of the GPU; neither is inside the timed
+interval, a pair of CUDA events on the launching stream around the step.
 
 The same step as the five separate C calls is timed afterwards (secondary
 numbers, with the sparse decode kernel bracketed alone).
@@ -66,6 +73,11 @@ def parse():
     p.add_argument("--prefill-batch", type=int, default=4, help="sequences of the prefill measurement")
     p.add_argument("--config-steps", type=int, default=100,
                    help="timed fused steps of each other decode workload (large block, ragged, sweep; 0: skip)")
+    p.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
+                   help="cold inputs by rotating over independent input sets, or by a 256 MiB memset per step")
+    p.add_argument("--sets", type=int, default=6, help="input sets of the rotation")
+    p.add_argument("--flush-steps", type=int, default=300,
+                   help="timed steps of the secondary memset-flush measurement of the headline (0: skip)")
     return p.parse_args()
 
 
@@ -315,21 +327,23 @@ OTHER_WORKLOADS = ["large_block", "ragged"] + SWEEP
 def other_configs(args, dev, world, peak, flush, stream):
     """The fused step on every other decode workload of the benchmark (same timing method as the
     headline), each with its algorithmic bytes and roofline fraction; each sweep batch also gets this
-    build's dense decode (sparse decode + combine over every block) beside it."""
+    build's dense decode (sparse decode + combine over every block, after a memset flush) beside it."""
     import torch
 
     from block_sparse_attention_seer_b200 import api
     from block_sparse_attention_seer_b200 import workloads as W
 
-    def timed(fn, n):
+    def timed(fns, n, rotate):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
-        for k in range(n + 5):
-            flush.zero_()
+        for k in range(n + 5 * len(fns)):
+            if not rotate:
+                flush.zero_()
             torch.cuda._sleep(300_000)
-            e = evs[k - 5] if k >= 5 else None
+            kk = k - 5 * len(fns)
+            e = evs[kk] if kk >= 0 else None
             if e:
                 e[0].record(stream)
-            fn()
+            fns[k % len(fns)]()
             if e:
                 e[1].record(stream)
         torch.cuda.synchronize()
@@ -344,10 +358,18 @@ def other_configs(args, dev, world, peak, flush, stream):
         lens = inp["seq_lens_host"]
         entry = {"kept_fraction_target": None}
         if not name.endswith("_dense"):
-            st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
-            st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
-            us = timed(lambda: st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"],
-                                             inp["seq_lens"]), args.config_steps)
+            rot = args.l2 == "rotate"
+            group = []  # the rotation's input sets (the first is `inp`), the same lengths
+            for k in range(max(1, args.sets) if rot else 1):
+                ik = inp if k == 0 else W.make_inputs(wl, seed=args.seed + rank + 1000 * k, device=dev,
+                                                      seq_lens=lens)
+                sk = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
+                sk.build_pool(ik["k_cache"], ik["w_k"], ik["seq_lens"])
+                group.append((ik, sk))
+            fns = [lambda i=i, s_=s_: s_.fused_step(i["q"], i["k_cache"], i["v_cache"], i["w_q"], i["w_k"],
+                                                    i["seq_lens"]) for i, s_ in group]
+            us = timed(fns, args.config_steps, rot)
+            st = group[0][1]
             step_bytes, _, toks, blocks = algorithmic_bytes(wl, lens, st.block_idx.cpu().numpy(),
                                                             st.num_selected.cpu().numpy())
             entry = {"us": round(us, 3), "bytes": step_bytes, "kept_blocks": blocks,
@@ -356,15 +378,15 @@ def other_configs(args, dev, world, peak, flush, stream):
                      "frac": round(step_bytes / (us * 1e-6) / 1e9 / peak, 4),
                      "frac_of_8tbs": round(step_bytes / (us * 1e-6) / 8e12, 4),
                      "kernel": "decode_step_kernel (the whole step)"}
-            del st
+            del st, group, fns
         else:  # this build's dense flash-decode at all blocks selected
             st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
             nbm = wl.nb_max
             idx_d, ns_d = W.identity_block_list(lens, wl.num_kv_heads, wl.block_size, nbm)
             idx_d = torch.from_numpy(idx_d).to(dev)
             ns_d = torch.from_numpy(ns_d).to(dev)
-            us = timed(lambda: st.attend(inp["q"], inp["k_cache"], inp["v_cache"], inp["seq_lens"], idx_d, ns_d,
-                                         nbm), max(10, args.config_steps // 4))
+            us = timed([lambda: st.attend(inp["q"], inp["k_cache"], inp["v_cache"], inp["seq_lens"], idx_d, ns_d,
+                                          nbm)], max(10, args.config_steps // 4), False)
             _, dense_bytes, toks, _ = algorithmic_bytes(wl, lens, idx_d.cpu().numpy(), ns_d.cpu().numpy())
             entry = {"us": round(us, 3), "bytes": dense_bytes, "gbs": round(dense_bytes / (us * 1e-6) / 1e9, 1),
                      "frac": round(dense_bytes / (us * 1e-6) / 1e9 / peak, 4),
@@ -404,61 +426,75 @@ def run_ours(args):
     wl = W.WORKLOADS[args.workload]
     if args.batch:
         wl = wl.with_(batch=args.batch, name=f"{wl.name}_batch{args.batch}")
-    inp = W.make_inputs(wl, seed=args.seed + rank, device=dev)
-    st = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
-    st.build_pool(inp["k_cache"], inp["w_k"], inp["seq_lens"])
-    st.set_update_start(inp["seq_lens"])
+    # the input sets of the rotation: independent data, the same lengths (so the same bytes per step)
+    R = max(1, args.sets) if args.l2 == "rotate" else 1
+    sets = []
+    for k in range(R):
+        ik = W.make_inputs(wl, seed=args.seed + rank + 1000 * k, device=dev,
+                           seq_lens=sets[0][0]["seq_lens_host"] if sets else None)
+        sk = api.DecodeStep(**wl.dims(), budget_tokens=wl.budget_tokens, device=dev)
+        sk.build_pool(ik["k_cache"], ik["w_k"], ik["seq_lens"])
+        sk.set_update_start(ik["seq_lens"])
+        sets.append((ik, sk, sk.parts(sk.num_splits)))
+    inp, st, _ = sets[0]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def run_fused():
-        st.fused_step(inp["q"], inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
+    def run_fused(k):
+        i, s_, _ = sets[k % R]
+        s_.fused_step(i["q"], i["k_cache"], i["v_cache"], i["w_q"], i["w_k"], i["seq_lens"])
 
-    def run_gate_calls():
-        api.seer_kpool_update(st.dims, inp["k_cache"], inp["w_k"], inp["seq_lens"], st.upd_start, st.kpool)
-        api.seer_gate_scores(st.dims, inp["q"], inp["w_q"], st.kpool, inp["seq_lens"], st.scores)
-        api.seer_select_blocks(st.dims, st.scores, inp["seq_lens"], st.budget_tokens, st.block_idx,
-                               st.num_selected)
+    def run_gate_calls(k):
+        i, s_, _ = sets[k % R]
+        api.seer_kpool_update(s_.dims, i["k_cache"], i["w_k"], i["seq_lens"], s_.upd_start, s_.kpool)
+        api.seer_gate_scores(s_.dims, i["q"], i["w_q"], s_.kpool, i["seq_lens"], s_.scores)
+        api.seer_select_blocks(s_.dims, s_.scores, i["seq_lens"], s_.budget_tokens, s_.block_idx,
+                               s_.num_selected)
 
-    o_part, lse_part = st.parts(st.num_splits)
+    def run_decode(k):
+        i, s_, (o_part, lse_part) = sets[k % R]
+        api.seer_sparse_decode(s_.dims, i["q"], i["k_cache"], i["v_cache"], i["seq_lens"], s_.block_idx,
+                               s_.num_selected, s_.kmax, s_.num_splits, 0.0, o_part, lse_part)
 
-    def run_decode():
-        api.seer_sparse_decode(st.dims, inp["q"], inp["k_cache"], inp["v_cache"], inp["seq_lens"], st.block_idx,
-                               st.num_selected, st.kmax, st.num_splits, 0.0, o_part, lse_part)
+    def run_combine(k):
+        i, s_, (o_part, lse_part) = sets[k % R]
+        api.seer_combine(s_.dims, o_part, lse_part, s_.num_splits, s_.out, s_.lse)
 
-    def run_combine():
-        api.seer_combine(st.dims, o_part, lse_part, st.num_splits, st.out, st.lse)
-
-    def prepare():
+    def prepare_flush():
         flush.zero_()
         torch.cuda._sleep(300_000)  # ~0.15 ms: the host enqueues the step ahead of the GPU
 
-    def fused_once(evs=None):
-        prepare()
+    def prepare():  # before a step of the rotation (or, with --l2 flush, the memset)
+        if args.l2 == "flush":
+            flush.zero_()
+        torch.cuda._sleep(300_000)
+
+    def fused_once(k, evs=None, flushed=False):
+        (prepare_flush if flushed else prepare)()
         if evs:
             evs[0].record(stream)
-        run_fused()
+        run_fused(k)
         if evs:
             evs[1].record(stream)
 
-    def separate_once(evs=None):
+    def separate_once(k, evs=None):
         prepare()
         if evs:
             evs[0].record(stream)
-        run_gate_calls()
+        run_gate_calls(k)
         if evs:
             evs[1].record(stream)
-        run_decode()
+        run_decode(k)
         if evs:
             evs[2].record(stream)
-        run_combine()
+        run_combine(k)
         if evs:
             evs[3].record(stream)
 
-    st.set_update_start(inp["seq_lens"])
     for _ in range(args.warmup):
-        fused_once()
-        separate_once()
+        for k in range(R):
+            fused_once(k)
+            separate_once(k)
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(smi_index(local))
@@ -469,7 +505,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for k in range(args.steps):
-        fused_once(ev[k])
+        fused_once(k, ev[k])
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     if world > 1:
@@ -478,11 +514,24 @@ def run_ours(args):
     step_ms = np.array([e[0].elapsed_time(e[1]) for e in ev])
     ms_step = float(step_ms.mean())
 
+    # secondary: the headline step on one input set with a 256 MiB memset before each step
+    flushed = None
+    if args.flush_steps > 0 and args.l2 == "rotate":
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.flush_steps)]
+        for k in range(args.flush_steps + 3):
+            fused_once(0, fev[k - 3] if k >= 3 else None, flushed=True)
+        torch.cuda.synchronize()
+        flush_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in fev]))
+        if world > 1:
+            (flush_ms,) = max_over_ranks([flush_ms], dev)
+        flushed = {"us": round(flush_ms * 1e3, 3), "steps": args.flush_steps,
+                   "method": "one input set, 256 MiB memset before every step (evicts the code too)"}
+
     # the same step as five separate calls (secondary: per-kernel brackets)
     n_sep = min(args.steps, 300)
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_sep)]
     for k in range(n_sep):
-        separate_once(sev[k])
+        separate_once(k, sev[k])
     torch.cuda.synchronize()
     sep_step_ms = float(np.mean([e[0].elapsed_time(e[3]) for e in sev]))
     ms_dec = float(np.mean([e[1].elapsed_time(e[2]) for e in sev]))
@@ -491,6 +540,7 @@ def run_ours(args):
         ms_step, ms_dec, sep_step_ms = max_over_ranks([ms_step, ms_dec, sep_step_ms], dev)
 
     lens = inp["seq_lens_host"]
+    sets_bytes = sum(t.numel() * t.element_size() for i, _, _ in sets for t in i.values() if torch.is_tensor(t))
     bidx = st.block_idx.cpu().numpy()
     nsel = st.num_selected.cpu().numpy()
     step_bytes, dec_bytes, toks, blocks = algorithmic_bytes(wl, lens, bidx, nsel)
@@ -501,6 +551,9 @@ def run_ours(args):
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "kernel": "decode_step_kernel",
                 "traffic": (traffic["dram_bytes_per_launch"] if traffic else None),
                 "algorithmic_bytes_per_launch": step_bytes}
+    if flushed:
+        flushed["gbs"] = round(step_bytes / (flushed["us"] * 1e-6) / 1e9, 1)
+        flushed["frac"] = round(step_bytes / (flushed["us"] * 1e-6) / 1e9 / peak, 4)
     dec_achieved = dec_bytes / (ms_dec * 1e-3) / 1e9
     separate = {"step_us": round(sep_step_ms * 1e3, 3), "launches_per_step": 5,
                 "gate_select_us": round(float(gate_ms.mean()) * 1e3, 3),
@@ -518,7 +571,7 @@ def run_ours(args):
         ns_d = torch.from_numpy(ns_d).to(dev)
         d_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.dense_steps)]
         for k in range(args.dense_steps + 3):
-            prepare()
+            prepare_flush()
             evs = d_ev[k - 3] if k >= 3 else None
             if evs:
                 evs[0].record(stream)
@@ -544,7 +597,7 @@ def run_ours(args):
         mlse_buf = torch.empty(wl.batch, wl.num_q_heads, dtype=torch.float32, device=dev)
         m_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.mass_steps)]
         for k in range(args.mass_steps + 3):
-            prepare()
+            prepare_flush()
             evs = m_ev[k - 3] if k >= 3 else None
             if evs:
                 evs[0].record(stream)
@@ -567,7 +620,7 @@ def run_ours(args):
         def timed(fn):
             v_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.variant_steps)]
             for k in range(args.variant_steps + 3):
-                prepare()
+                prepare_flush()
                 evs = v_ev[k - 3] if k >= 3 else None
                 if evs:
                     evs[0].record(stream)
@@ -617,7 +670,7 @@ def run_ours(args):
         for name, fn in calls.items():
             p_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.prefill_steps)]
             for kk in range(args.prefill_steps + 1):
-                prepare()
+                prepare_flush()
                 evs = p_ev[kk - 1] if kk >= 1 else None
                 if evs:
                     evs[0].record(stream)
@@ -648,9 +701,12 @@ def run_ours(args):
         nq, nkv = B * Hq * D, B * Hkv * D
         last = torch.from_numpy(np.maximum(lens.astype(np.int64) - 1, 0)).to(dev)
         rows_b = torch.arange(B, device=dev)
-        kn = inp["k_cache"][rows_b, :, last, :]  # the token already in the cache: the step is unchanged
-        vn = inp["v_cache"][rows_b, :, last, :]
-        packed_h = torch.cat([inp["q"].reshape(-1), kn.reshape(-1), vn.reshape(-1)]).cpu().pin_memory()
+        packed = []
+        for i, _, _ in sets:
+            kn = i["k_cache"][rows_b, :, last, :]  # the token already in the cache: the step is unchanged
+            vn = i["v_cache"][rows_b, :, last, :]
+            packed.append(torch.cat([i["q"].reshape(-1), kn.reshape(-1), vn.reshape(-1)]).cpu().pin_memory())
+        packed_h = packed[0]
         stage = torch.empty_like(packed_h, device=dev)
         q_d = stage[:nq].view(B, Hq, D)
         kn_d = stage[nq:nq + nkv].view(B, Hkv, D)
@@ -660,15 +716,15 @@ def run_ours(args):
         d2h = out_h.numel() * 2
         e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
         for k in range(args.e2e_steps + 5):
-            flush.zero_()
-            torch.cuda._sleep(300_000)
+            prepare()
             evs = e_ev[k - 5] if k >= 5 else None
+            i, s_, _ = sets[k % R]
             if evs:
                 evs[0].record(stream)
-            stage.copy_(packed_h, non_blocking=True)
-            api.seer_append_kv(st.dims, kn_d, vn_d, inp["seq_lens"], inp["k_cache"], inp["v_cache"])
-            st.fused_step(q_d, inp["k_cache"], inp["v_cache"], inp["w_q"], inp["w_k"], inp["seq_lens"])
-            out_h.copy_(st.out, non_blocking=True)
+            stage.copy_(packed[k % R], non_blocking=True)
+            api.seer_append_kv(s_.dims, kn_d, vn_d, i["seq_lens"], i["k_cache"], i["v_cache"])
+            s_.fused_step(q_d, i["k_cache"], i["v_cache"], i["w_q"], i["w_k"], i["seq_lens"])
+            out_h.copy_(s_.out, non_blocking=True)
             if evs:
                 evs[1].record(stream)
         torch.cuda.synchronize()
@@ -701,12 +757,15 @@ def run_ours(args):
                        "kept_blocks": blocks, "kept_tokens": toks,
                        "sparsity": round(1 - toks / float(sum(int(x) for x in lens) * wl.num_kv_heads), 4),
                        "parallelism": f"replicas x{world}",
-                       "l2": "256 MiB memset before every step, outside the timed interval",
+                       "l2": (f"inputs larger than L2: steps rotate over {R} independent input sets "
+                              f"({sets_bytes / 2**30:.1f} GiB), no flush" if args.l2 == "rotate" else
+                              "256 MiB memset before every step, outside the timed interval"),
                        "timing": "CUDA events per step on the launching stream; mean over steps; max over ranks"},
             "step_bytes": step_bytes,
             "step_hbm_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
             "step_frac_of_8tbs": round(step_bytes / (ms_step * 1e-3) / 8e12, 4),
             "step_us_p50": round(float(np.median(step_ms)) * 1e3, 3),
+            "l2_flush": flushed,
             "separate_calls": separate,
             "dense_baseline": dense,
             "block_mass": block_mass,

@@ -233,6 +233,14 @@ struct SelectBins {
     }
 };
 
+// Called once by every thread of select_row when the first histogram has
+// fixed the threshold bin: every candidate whose bin (under `bins`, over the
+// full key range) is above `bstar` is kept, whatever the rest of the search
+// finds. The default does nothing.
+struct NoThreshold {
+    __device__ __forceinline__ void operator()(const SelectBins&, int) const {}
+};
+
 // Block list of one row. keys[0 .. NB-2] (shared memory) hold the order keys
 // of the candidate blocks 0 .. NB-2. Writes the kept indices in ascending
 // order to out[0 .. kb-1] (kb = min(kmax, NB): block NB-1 always, plus the
@@ -250,9 +258,10 @@ struct SelectBins {
 // range of one key value keeps its lowest indices. The common case is a
 // single histogram and seven barriers.
 
-template <int kThreads>
+template <int kThreads, typename OnThreshold = NoThreshold>
 __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __restrict__ out,
-                           SelectSmem<kThreads>& sm, int32_t* head = nullptr) {
+                           SelectSmem<kThreads>& sm, int32_t* head = nullptr,
+                           OnThreshold on_threshold = OnThreshold()) {
     constexpr int kWarps = kThreads / 32;
     constexpr unsigned kFull = 0xffffffffu;
     constexpr int kBinsPer = (kSelectBins + kThreads - 1) / kThreads;
@@ -318,6 +327,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
     int rem = m;  // how many of the keys inside [lo, hi] are kept
     uint32_t kT;
     int iT;
+    bool first_pass = true;
     while (true) {
         if (lo == hi) {  // one key value left: its rem lowest indices
             int c = 0;
@@ -363,6 +373,8 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
         __syncthreads();
         const int bstar = sm.bstar, bcount = sm.bcount;
         rem -= sm.above;
+        if (first_pass) on_threshold(bins, bstar);  // [lo, hi] is still the full key range
+        first_pass = false;
         if (bcount <= kSelectBucket) {
             // gather the bin, then rank each entry against the others: T has rank rem - 1
             for (int i = tid; i < ncand; i += kThreads) {

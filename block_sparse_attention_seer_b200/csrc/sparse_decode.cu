@@ -617,6 +617,7 @@ struct StepParams {
     int chunk;                               // list positions per claim from the front
     int keys_off, chunk_off, n_gate_stages;  // gate keys and pooled-key copies inside the stage ring
     int wq_stages;                           // rows fit the grid: the last gate stages first hold W_q
+    int n_early;                             // one CTA per row: decode stages issued during the selection
     int sel_off;                             // rows this CTA selected (shared memory, kMaxSelRows)
     int refresh_off;                         // pool scratch of the helper warps (outside the ring)
 };
@@ -685,24 +686,39 @@ struct SelList {
     int count;
     int publish;  // rows fit the grid: the row this CTA selected, released after the gate (else -1)
     int own_len;  // rows fit the grid: the length of the row this CTA gated
+    int early_count;            // one CTA per row: stages the gate issued during the selection
+    int early_ids[kMaxStages];  // their blocks (certainly kept), ascending
     int row[kMaxSelRows];
     int nsel[kMaxSelRows];
     int len[kMaxSelRows];
     int head[kMaxSelRows][kSelectHead];  // the first list entries of each
 };
 
+// The gate's scratch (in the merge area). Once a batch is scored only rows and
+// last_of are read again: the selection's scratch overlays what precedes them
+// (the padding makes room for it where the query arrays are smaller).
+template <int D, int DG>
+constexpr int gate_work_bytes() {
+    return 4 * (kMaxBatchRows * D + kMaxBatchRows * DG + DG) + (int)sizeof(PoolSmem<D>);
+}
 template <int D, int DG>
 struct GateScratch {
     alignas(16) float qbar[kMaxBatchRows][D];
     alignas(16) float qg[kMaxBatchRows][DG];
     alignas(16) float kp_new[DG];
     PoolSmem<D> pool;
+    unsigned char pad[(int)sizeof(SelectSmem<kStepThreads>) > gate_work_bytes<D, DG>()
+                          ? (int)sizeof(SelectSmem<kStepThreads>) - gate_work_bytes<D, DG>() + 16
+                          : 16];
     GateRow rows[kMaxBatchRows];
     int last_of[kMaxBatchRows];
 };
 static_assert(sizeof(GateScratch<128, 128>) <= kGateScratchBytes, "gate scratch");
-static_assert(sizeof(SelectSmem<kStepThreads>) <= kGateChunkBytes, "the select scratch reuses a chunk stage");
 static_assert(sizeof(GateScratch<64, 128>) <= kGateScratchBytes, "gate scratch");
+static_assert(sizeof(GateScratch<64, 64>) <= kGateScratchBytes, "gate scratch");
+using GateScratchSmallest = GateScratch<64, 64>;
+static_assert(offsetof(GateScratchSmallest, rows) >= sizeof(SelectSmem<kStepThreads>),
+              "the selection's scratch before the gate rows");
 
 // The gate. The R x NBmax pooled-key positions (row-major, the layout of
 // kpool) are cut into gate_ctas equal contiguous ranges (with rows <= SMs,
@@ -717,7 +733,8 @@ static_assert(sizeof(GateScratch<64, 128>) <= kGateScratchBytes, "gate scratch")
 // are refreshed here. `old_ctr` (the launch counter before this CTA's add) is
 // valid in thread 0.
 template <int D, int BLK, int DG>
-__device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, unsigned long long old_ctr) {
+__device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const Params& p, const StepParams& f,
+                           const Smem& m, unsigned long long old_ctr) {
     constexpr int kThreads = kStepThreads;
     constexpr int kWarps = kThreads / 32;
     constexpr int kChunkRows = kGateChunkBytes / (DG * 4);
@@ -958,7 +975,7 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
         }
         __syncthreads();
         // the rows this CTA completes: load their keys, then the CTA selects each
-        SelectSmem<kThreads>& ssm = *reinterpret_cast<SelectSmem<kThreads>*>(m.base + f.chunk_off);
+        SelectSmem<kThreads>& ssm = *reinterpret_cast<SelectSmem<kThreads>*>(m.merge);  // over the query arrays
         SelList& sel = *reinterpret_cast<SelList*>(m.base + f.sel_off);
         for (int k = 0; k < nb; ++k) {
             if (!sm.last_of[k]) continue;
@@ -988,8 +1005,57 @@ __device__ void gate_phase(const Params& p, const StepParams& f, const Smem& m, 
                 }
             }
             __syncthreads();
-            select_row<kThreads>(keys, g.NB, p.kmax, f.block_idx + (size_t)g.r * p.kmax, ssm,
-                                 si < kMaxSelRows ? sel.head[si] : nullptr);
+            int32_t* list = f.block_idx + (size_t)g.r * p.kmax;
+            int32_t* head = si < kMaxSelRows ? sel.head[si] : nullptr;
+            if (whole_rows && f.n_early > 0 && kb > 0) {
+                // One CTA per row: once the first histogram fixes the threshold bin, the
+                // producer warp starts the decode on the first candidates above it (kept
+                // whatever the rest of the search finds) while the others finish the list.
+                const int ncand = g.NB - 1;
+                auto early = [&](const SelectBins& bins, int bstar) {
+                    if (warp != kConsumerWarps) return;
+                    using C = Cfg<D, BLK>;
+                    constexpr unsigned kFull = 0xffffffffu;
+                    const uint64_t policy = l2_policy_evict_first();
+                    const uint32_t qbytes = (uint32_t)(p.G * D * 2);
+                    int n = 0;
+                    for (int i0 = 0; i0 < ncand && n < f.n_early; i0 += 32) {
+                        const int i = i0 + lane;
+                        unsigned msk = __ballot_sync(kFull, i < ncand && bins(keys[i]) > bstar);
+                        while (msk != 0u && n < f.n_early) {
+                            const int j = i0 + __ffs(msk) - 1;  // a full block: j < NB - 1
+                            msk &= msk - 1u;
+                            if (lane == 0) {  // stage n of a fresh ring: its empty phase has passed
+                                int* sinfo = m.sinfo + n * kStageInfoWords;
+                                sinfo[0] = BLK;
+                                sinfo[1] = g.r;
+                                sinfo[2] = n == 0 ? kRunStart : 0;
+                                sinfo[3] = 0;
+                                sinfo[4] = n + 1;
+                                sinfo[5] = kb;
+                                const uint32_t fb = m.full(n);
+                                mbar_arrive_expect_tx(fb, 2u * C::kTileBytes + (n == 0 ? qbytes : 0u));
+                                const uint32_t stK = m.sbase + (uint32_t)n * p.stage_bytes;
+                                const int y = g.r * p.Lmax + j * BLK;
+#pragma unroll
+                                for (int bx = 0; bx < C::kBoxes; ++bx) {
+                                    tma_load_2d(stK + bx * C::kBoxBytes, tmK, fb, bx * 64, y, policy);
+                                    tma_load_2d(stK + C::kTileBytes + bx * C::kBoxBytes, tmV, fb, bx * 64, y, policy);
+                                }
+                                if (n == 0)
+                                    bulk_load(stK + 2 * C::kTileBytes,
+                                              p.q + ((size_t)g.b * p.Hq + (size_t)g.kvh * p.G) * D, qbytes, fb);
+                                sel.early_ids[n] = j;
+                            }
+                            ++n;
+                        }
+                    }
+                    if (lane == 0) sel.early_count = n;
+                };
+                select_row<kThreads>(keys, g.NB, p.kmax, list, ssm, head, early);
+            } else {
+                select_row<kThreads>(keys, g.NB, p.kmax, list, ssm, head);
+            }
             if (kb == 0) {  // a row without tokens is written here
                 const size_t head0 = (size_t)g.b * p.Hq + (size_t)g.kvh * p.G;
                 for (int i = tid; i < p.G * D; i += kThreads) f.out[head0 * D + i] = __float2bfloat16(0.f);
@@ -1098,7 +1164,10 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
 
     // Stream one run of `row` (nsel list positions) from the piece [a0, a1) it holds;
     // from the front, further pieces are claimed one ahead until the row has none left.
-    auto run = [&](int row, int nsel, int a0, int a1, bool from_front, const int* head, int fixed_slot, int Lrow) {
+    // `ne` > 0: stages 0 .. ne-1 were issued by the gate (blocks sel.early_ids,
+    // the run's start); those blocks are skipped here (never the list's last).
+    auto run = [&](int row, int nsel, int a0, int a1, bool from_front, const int* head, int fixed_slot, int Lrow,
+                   int ne) {
         const int b = row / p.Hkv;
         const int L = Lrow >= 0 ? Lrow : clamp_len(p.seq_lens[b], p.Lmax);
         const int NB = (L + BLK - 1) / BLK;
@@ -1116,8 +1185,9 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
         __syncwarp();
         int wbase = a0;  // the lanes hold list[wbase + lane]; a list this CTA selected starts in shared memory
         int jl = head ? head[lane] : ((a0 + lane < p.kmax) ? __ldcg(list + a0 + lane) : -1);
+        const int early_id = lane < ne ? sel.early_ids[lane] : -1;
         int nrun = 0;
-        bool first = true;
+        bool first = ne == 0;
         while (ok) {
             const int cnt = a1 - a0;
             int na0 = 0, na1 = 0;
@@ -1128,6 +1198,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
                     jl = (pos + lane < p.kmax) ? __ldcg(list + pos + lane) : -1;
                 }
                 const int j = __shfl_sync(kFull, jl, pos - wbase);
+                if (ne > 0 && k + 1 < cnt && __any_sync(kFull, early_id == j)) continue;
                 const int valid = (j >= 0 && j < NB) ? min(BLK, L - j * BLK) : 0;
                 int flags = first ? kRunStart : 0;
                 if (k + 1 == cnt) {  // the run goes on with the claim in flight, if it took anything
@@ -1187,7 +1258,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
         a0 = __shfl_sync(kFull, a0, 0);
         a1 = __shfl_sync(kFull, a1, 0);
         nsel = __shfl_sync(kFull, nsel, 0);
-        if (a0 < a1) run(row, nsel, a0, a1, true, nullptr, -1, -1);
+        if (a0 < a1) run(row, nsel, a0, a1, true, nullptr, -1, -1, 0);
     };
 
     const int nselrows = sel.count;
@@ -1216,7 +1287,11 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
                 // a fixed slot per non-empty part: the merge adds the parts in the same
                 // order on every call, so the output is the same bit for bit
                 const int slot = nsel >= f.gate_cpr ? part : a0;
-                if (a0 < a1) run(row, nsel, a0, a1, false, a0 == 0 ? head : nullptr, slot, sel.own_len);
+                // one CTA per row: the gate may have issued the first stages already
+                const int ne = f.gate_cpr == 1 ? sel.early_count : 0;
+                st = ne;  // < nst: the ring has not wrapped
+                issued = ne;
+                if (a0 < a1) run(row, nsel, a0, a1, false, a0 == 0 ? head : nullptr, slot, sel.own_len, ne);
             }
         }
         if (ok) put(0, 0, 0, kExit, 0, 0, 0, false);
@@ -1232,7 +1307,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
     // ---- rows outnumber the CTAs:
     // ---- 1. the rows this CTA selected, from the chunk it kept
     for (int i = 0; ok && i < nselrows; ++i)
-        run(sel.row[i], sel.nsel[i], 0, min(chunk, sel.nsel[i]), true, sel.head[i], -1, sel.len[i]);
+        run(sel.row[i], sel.nsel[i], 0, min(chunk, sel.nsel[i]), true, sel.head[i], -1, sel.len[i], 0);
 
     // ---- 2. its other home rows
     int home_lo, home_hi;
@@ -1290,7 +1365,7 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
             a0 = __shfl_sync(kFull, a0, 0);
             a1 = __shfl_sync(kFull, a1, 0);
             nsel = __shfl_sync(kFull, nsel, 0);
-            if (a0 < a1) run(row, nsel, a0, a1, false, nullptr, -1, -1);
+            if (a0 < a1) run(row, nsel, a0, a1, false, nullptr, -1, -1, 0);
             empty_windows = 0;
             idle_since = 0;
             continue;  // look at the same window again
@@ -1526,8 +1601,9 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         SelList& sel = *reinterpret_cast<SelList*>(m.base + f.sel_off);
         sel.count = 0;
         sel.publish = -1;
+        sel.early_count = 0;
     }
-    gate_phase<D, BLK, DG>(p, f, m, old_ctr);
+    gate_phase<D, BLK, DG>(&tmK, &tmV, p, f, m, old_ctr);
     fence_proxy_async_smem();  // the gate's use of the ring precedes the decode's copies into it
     if (threadIdx.x == 0) {
         const uint32_t epoch = epoch_of(old_ctr);
@@ -1733,9 +1809,12 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     f.dg = s.dg;
     f.refresh_off = l.refresh_off;
     f.sel_off = l.sel_off;
-    f.keys_off = 0;
-    f.chunk_off = keys_bytes;
+    f.keys_off = ring - keys_bytes;  // the gate's order keys end the ring: the early stages start at its front
+    f.chunk_off = 0;
     f.n_gate_stages = n_gate > kMaxGateStages ? kMaxGateStages : n_gate;
+    // one CTA per row: decode stages that fit before the keys may start during the selection
+    const int n_early = f.keys_off / l.stage_bytes < l.nst - 1 ? f.keys_off / l.stage_bytes : l.nst - 1;
+    f.n_early = geo.gate_cpr == 1 ? n_early : 0;
     // rows fit the grid: W_q of the row's head (dg x D fp32) first fills the last gate stages
     const int wq_st = (DG * D * 4 + kGateChunkBytes - 1) / kGateChunkBytes;
     f.wq_stages = (geo.gate_cpr > 0 && f.n_gate_stages > wq_st) ? wq_st : 0;

@@ -315,7 +315,9 @@ seer_status seer_append_kv(const seer_dims* dims, const void* k_new, const void*
  * block lists); the CTA that completes a row's gate publishes the row (a
  * release flag). The decode of a row starts as soon as it is published: when
  * rows fit the grid, the CTAs that gated a row stream even, fixed parts of its
- * kept list (a row held by one CTA is written straight to out); when rows
+ * kept list (a row held by one CTA is written straight to out, and its first
+ * blocks, those the selection keeps whatever the rest of its search finds,
+ * start streaming before the list is complete); when rows
  * outnumber the CTAs, CTAs take pieces of each list from the front and help
  * with the rows that have most left from the back. The CTA that completes a
  * row's positions merges its partial results into out / lse_out as

@@ -326,7 +326,11 @@ def test_shared_memory_layout_fits(D, blk, G):
                 n_gate = (ring - keys) // GATE_CHUNK
                 assert n_gate >= 1  # at least one pooled-key copy in flight
                 n_gate = min(n_gate, MAX_GATE_STAGES)
-                assert keys + n_gate * GATE_CHUNK <= ring
+                keys_off = ring - keys  # the order keys end the ring; pooled-key copies start at 0
+                assert keys_off % 1024 == 0 and n_gate * GATE_CHUNK <= keys_off
+                # one CTA per row: decode stages issued during the selection stay clear of the keys
+                n_early = min(keys_off // l["stage"], l["nst"] - 1)
+                assert 0 <= n_early <= MAX_STAGES - 1 and n_early * l["stage"] <= keys_off
                 for dg in (64, 128):
                     # rows that fit the grid: W_q (dg x D fp32, one bulk copy) first fills the
                     # last wq gate stages, used only when at least one stage stays free for keys
