@@ -387,8 +387,9 @@ class Bins:
         return ((k - self.lo) & 0xffffffff) >> self.shift
 
 
-def select_row(keys, NB, kmax, T):
-    """select_row with T threads: every read of keys / hist / bucket and write of out is checked."""
+def select_row(keys, NB, kmax, T, on_threshold=None):
+    """select_row with T threads: every read of keys / hist / bucket and write of out is checked.
+    on_threshold(bins, bstar) is called once, when the first histogram has fixed the threshold bin."""
     def K(i):
         assert 0 <= i < NB - 1 <= len(keys), ("keys", i)
         return keys[i]
@@ -458,6 +459,9 @@ def select_row(keys, NB, kmax, T):
         assert found is not None
         bstar, bcount, above = found
         rem -= above
+        if on_threshold is not None:
+            on_threshold(b, bstar)
+            on_threshold = None
         assert 1 <= rem <= bcount
         if bcount <= BUCKET:
             bucket = [(K(i), i) for i in range(ncand) if lo <= K(i) <= hi and b(K(i)) == bstar]
@@ -517,6 +521,34 @@ SCORE_FAMILIES = {
     "ulps": lambda rng, n: np.where(rng.random(n) < 0.02, 1e30, 1.0 + rng.integers(0, 3 * n, n) * 2.0 ** -23),
     "inf_nan": lambda rng, n: rng.choice([np.inf, -np.inf, np.nan, 1.0, -3e38, 3e38, 0.5], n),
 }
+
+
+@pytest.mark.parametrize("NB,kmax", [(33, 8), (64, 8), (512, 64), (512, 2), (1024, 103), (1025, 300), (4096, 64)])
+def test_early_stages_take_only_kept_blocks_and_the_rest_completes_the_list(NB, kmax):
+    """The fused step (one CTA per row) issues its first decode stages from the candidates whose
+    bin lies above the first histogram's threshold bin, in index order, before the selection has
+    finished; its producer later walks the finished list and skips those blocks. Every such block
+    must be kept, never the open last block, and the stages issued plus the ones walked must be the
+    kept list exactly once each."""
+    rng = np.random.default_rng(NB * 7 + kmax)
+    for name, gen in SCORE_FAMILIES.items():
+        with np.errstate(all="ignore"):
+            f = gen(rng, NB - 1).astype(np.float32)
+        keys = [order_key(x) for x in f] + [0]
+        for n_early in (1, 5, 7):
+            early = []
+
+            def hook(b, bstar):
+                for i in range(NB - 1):  # the producer warp's ascending scan, 32 candidates a ballot
+                    if len(early) < n_early and b(keys[i]) > bstar:
+                        early.append(i)
+            out = select_row(keys, NB, kmax, 384, hook)
+            kept = [j for j in out if j >= 0]
+            assert kept == sorted_selection(keys, NB, kmax)[:len(kept)], name
+            assert len(early) <= n_early and early == sorted(set(early))
+            assert all(j in kept and j != NB - 1 for j in early), (name, early)
+            walked = [j for k, j in enumerate(kept) if not (k + 1 < len(kept) and j in early)]
+            assert sorted(early + walked) == kept and walked[-1] == NB - 1, name
 
 
 @pytest.mark.parametrize("NB,kmax,T", [(1, 8, 256), (2, 1, 256), (2, 8, 384), (33, 8, 384), (512, 64, 384),
