@@ -246,9 +246,9 @@ struct NoThreshold {
 // order to out[0 .. kb-1] (kb = min(kmax, NB): block NB-1 always, plus the
 // kb-1 largest keys, equal keys going to the lower index) and -1 to out[kb ..
 // kmax). When `head` is given (shared memory, kSelectHead entries), the first
-// kSelectHead entries of the list are written there too. Every thread of the
-// CTA calls it; shared memory is reused only after a barrier that follows the
-// call.
+// kSelectHead entries of the list are written there too. Threads 0 ..
+// kThreads-1 call it and meet at `sync` (by default the whole CTA); shared
+// memory is reused only after a barrier that follows the call.
 //
 // T is found by narrowing a key range [lo, hi] known to hold it: a histogram
 // of the range (SelectBins), a CTA scan of the bins from the top to the bin
@@ -258,10 +258,10 @@ struct NoThreshold {
 // range of one key value keeps its lowest indices. The common case is a
 // single histogram and seven barriers.
 
-template <int kThreads, typename OnThreshold = NoThreshold>
+template <int kThreads, typename OnThreshold = NoThreshold, typename Sync = CtaSync>
 __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __restrict__ out,
                            SelectSmem<kThreads>& sm, int32_t* head = nullptr,
-                           OnThreshold on_threshold = OnThreshold()) {
+                           OnThreshold on_threshold = OnThreshold(), Sync sync = Sync()) {
     constexpr int kWarps = kThreads / 32;
     constexpr unsigned kFull = 0xffffffffu;
     constexpr int kBinsPer = (kSelectBins + kThreads - 1) / kThreads;
@@ -302,7 +302,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
             sm.wlo[warp] = a;
             sm.whi[warp] = b;
         }
-        __syncthreads();
+        sync();
         glo = __reduce_min_sync(kFull, lane < kWarps ? sm.wlo[lane] : 0xffffffffu);
         ghi = __reduce_max_sync(kFull, lane < kWarps ? sm.whi[lane] : 0u);
     };
@@ -310,7 +310,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
     auto block_scan = [&](int v, int& total) {
         const int x = warp_inclusive_scan(v);
         if (lane == 31) sm.wsum[warp] = x;
-        __syncthreads();
+        sync();
         const unsigned w = lane < kWarps ? (unsigned)sm.wsum[lane] : 0u;
         total = (int)__reduce_add_sync(kFull, w);
         return (int)__reduce_add_sync(kFull, lane < warp ? w : 0u) + x - v;
@@ -339,7 +339,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
                 for (int i = c0; i < c1; ++i)
                     if (keys[i] == lo && ++seen == rem) sm.iT = i;
             }
-            __syncthreads();
+            sync();
             kT = lo;
             iT = sm.iT;
             break;
@@ -350,7 +350,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
             const uint32_t k = keys[i];
             if (k >= lo && k <= hi) atomicAdd(&sm.hist[bins(k)], 1);
         }
-        __syncthreads();
+        sync();
         int mine = 0;
 #pragma unroll
         for (int q = 0; q < kBinsPer; ++q)
@@ -370,7 +370,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
                 run += c;
             }
         }
-        __syncthreads();
+        sync();
         const int bstar = sm.bstar, bcount = sm.bcount;
         rem -= sm.above;
         if (first_pass) on_threshold(bins, bstar);  // [lo, hi] is still the full key range
@@ -385,7 +385,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
                     sm.bidx[at] = i;
                 }
             }
-            __syncthreads();
+            sync();
             if (tid < bcount) {
                 const uint32_t mk = sm.bkey[tid];
                 const int mi = sm.bidx[tid];
@@ -399,7 +399,7 @@ __device__ void select_row(const uint32_t* keys, int NB, int kmax, int32_t* __re
                     sm.iT = mi;
                 }
             }
-            __syncthreads();
+            sync();
             kT = sm.kT;
             iT = sm.iT;
             break;

@@ -143,6 +143,7 @@ struct Smem {
     __device__ __forceinline__ uint32_t gate(int st) const { return bars + 16u * nst + 8u + 8u * st; }
     __device__ __forceinline__ uint32_t helper() const { return bars + 16u * nst + 8u + 8u * kMaxGateStages; }
     __device__ __forceinline__ uint32_t wq() const { return bars + 16u * nst + 16u + 8u * kMaxGateStages; }
+    __device__ __forceinline__ uint32_t thr() const { return bars + 16u * nst + 24u + 8u * kMaxGateStages; }
 };
 
 __device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) {
@@ -163,6 +164,7 @@ __device__ __forceinline__ Smem setup_smem(unsigned char* raw, const Params& p) 
         for (int st = 0; st < kMaxGateStages; ++st) mbar_init(m.gate(st), 1);
         mbar_init(m.helper(), kHelperThreads / 32);
         mbar_init(m.wq(), 1);
+        mbar_init(m.thr(), 1);
         for (int i = 0; i < kInfoWords; ++i) m.info[i] = 0;
         fence_mbar_init();
     }
@@ -678,6 +680,12 @@ struct GateRow {
 };
 constexpr int kMaxBatchRows = 8;
 
+// The barrier of the selection's 352 threads (warps 0 .. 10) when the last
+// warp issues the first decode stages meanwhile; no other code uses id 1.
+struct SelectGroupSync {
+    __device__ __forceinline__ void operator()() const { named_barrier_sync(1, kStepThreads - 32); }
+};
+
 // Rows a CTA selected, kept for its decode producer (outside the stage ring):
 // the CTA keeps the first chunk of each of them, so it starts streaming with
 // no global round trip.
@@ -688,11 +696,15 @@ struct SelList {
     int own_len;  // rows fit the grid: the length of the row this CTA gated
     int early_count;            // one CTA per row: stages the gate issued during the selection
     int early_ids[kMaxStages];  // their blocks (certainly kept), ascending
+    int thr_valid;              // the selection's first threshold bin, for the warp that issues them
+    int thr_bstar;
+    SelectBins thr_bins;
     int row[kMaxSelRows];
     int nsel[kMaxSelRows];
     int len[kMaxSelRows];
     int head[kMaxSelRows][kSelectHead];  // the first list entries of each
 };
+static_assert(sizeof(SelectBins) == 20 && sizeof(SelList) == 4556, "the host-side replica of the layout");
 
 // The gate's scratch (in the merge area). Once a batch is scored only rows and
 // last_of are read again: the selection's scratch overlays what precedes them
@@ -1008,51 +1020,71 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
             int32_t* list = f.block_idx + (size_t)g.r * p.kmax;
             int32_t* head = si < kMaxSelRows ? sel.head[si] : nullptr;
             if (whole_rows && f.n_early > 0 && kb > 0) {
-                // One CTA per row: once the first histogram fixes the threshold bin, the
-                // producer warp starts the decode on the first candidates above it (kept
-                // whatever the rest of the search finds) while the others finish the list.
-                const int ncand = g.NB - 1;
-                auto early = [&](const SelectBins& bins, int bstar) {
-                    if (warp != kConsumerWarps) return;
-                    using C = Cfg<D, BLK>;
-                    constexpr unsigned kFull = 0xffffffffu;
-                    const uint64_t policy = l2_policy_evict_first();
-                    const uint32_t qbytes = (uint32_t)(p.G * D * 2);
+                // One CTA per row: once the first histogram fixes the threshold bin, every
+                // candidate above it is kept whatever the rest of the search finds. Warps
+                // 0 .. 10 select (meeting at a named barrier); the last warp waits for that
+                // bin and meanwhile starts the decode on the first such candidates.
+                constexpr int kSelThreads = kThreads - 32;
+                if (warp == kWarps - 1) {
+                    const bool got = mbar_wait(m.thr(), 0u);
+                    __syncwarp();
+                    if (!got) record_failure(m.info);
                     int n = 0;
-                    for (int i0 = 0; i0 < ncand && n < f.n_early; i0 += 32) {
-                        const int i = i0 + lane;
-                        unsigned msk = __ballot_sync(kFull, i < ncand && bins(keys[i]) > bstar);
-                        while (msk != 0u && n < f.n_early) {
-                            const int j = i0 + __ffs(msk) - 1;  // a full block: j < NB - 1
-                            msk &= msk - 1u;
-                            if (lane == 0) {  // stage n of a fresh ring: its empty phase has passed
-                                int* sinfo = m.sinfo + n * kStageInfoWords;
-                                sinfo[0] = BLK;
-                                sinfo[1] = g.r;
-                                sinfo[2] = n == 0 ? kRunStart : 0;
-                                sinfo[3] = 0;
-                                sinfo[4] = n + 1;
-                                sinfo[5] = kb;
-                                const uint32_t fb = m.full(n);
-                                mbar_arrive_expect_tx(fb, 2u * C::kTileBytes + (n == 0 ? qbytes : 0u));
-                                const uint32_t stK = m.sbase + (uint32_t)n * p.stage_bytes;
-                                const int y = g.r * p.Lmax + j * BLK;
+                    if (got && sel.thr_valid) {
+                        using C = Cfg<D, BLK>;
+                        constexpr unsigned kFull = 0xffffffffu;
+                        const SelectBins bins = sel.thr_bins;
+                        const int bstar = sel.thr_bstar;
+                        const int ncand = g.NB - 1;
+                        const uint64_t policy = l2_policy_evict_first();
+                        const uint32_t qbytes = (uint32_t)(p.G * D * 2);
+                        for (int i0 = 0; i0 < ncand && n < f.n_early; i0 += 32) {
+                            const int i = i0 + lane;
+                            unsigned msk = __ballot_sync(kFull, i < ncand && bins(keys[i]) > bstar);
+                            while (msk != 0u && n < f.n_early) {
+                                const int j = i0 + __ffs(msk) - 1;  // a full block: j < NB - 1
+                                msk &= msk - 1u;
+                                if (lane == 0) {  // stage n of a fresh ring: its empty phase has passed
+                                    int* sinfo = m.sinfo + n * kStageInfoWords;
+                                    sinfo[0] = BLK;
+                                    sinfo[1] = g.r;
+                                    sinfo[2] = n == 0 ? kRunStart : 0;
+                                    sinfo[3] = 0;
+                                    sinfo[4] = n + 1;
+                                    sinfo[5] = kb;
+                                    const uint32_t fb = m.full(n);
+                                    mbar_arrive_expect_tx(fb, 2u * C::kTileBytes + (n == 0 ? qbytes : 0u));
+                                    const uint32_t stK = m.sbase + (uint32_t)n * p.stage_bytes;
+                                    const int y = g.r * p.Lmax + j * BLK;
 #pragma unroll
-                                for (int bx = 0; bx < C::kBoxes; ++bx) {
-                                    tma_load_2d(stK + bx * C::kBoxBytes, tmK, fb, bx * 64, y, policy);
-                                    tma_load_2d(stK + C::kTileBytes + bx * C::kBoxBytes, tmV, fb, bx * 64, y, policy);
+                                    for (int bx = 0; bx < C::kBoxes; ++bx) {
+                                        tma_load_2d(stK + bx * C::kBoxBytes, tmK, fb, bx * 64, y, policy);
+                                        tma_load_2d(stK + C::kTileBytes + bx * C::kBoxBytes, tmV, fb, bx * 64, y,
+                                                    policy);
+                                    }
+                                    if (n == 0)
+                                        bulk_load(stK + 2 * C::kTileBytes,
+                                                  p.q + ((size_t)g.b * p.Hq + (size_t)g.kvh * p.G) * D, qbytes, fb);
+                                    sel.early_ids[n] = j;
                                 }
-                                if (n == 0)
-                                    bulk_load(stK + 2 * C::kTileBytes,
-                                              p.q + ((size_t)g.b * p.Hq + (size_t)g.kvh * p.G) * D, qbytes, fb);
-                                sel.early_ids[n] = j;
+                                ++n;
                             }
-                            ++n;
                         }
                     }
                     if (lane == 0) sel.early_count = n;
-                };
-                select_row<kThreads>(keys, g.NB, p.kmax, list, ssm, head, early);
+                } else {
+                    auto threshold = [&](const SelectBins& bins, int bstar) {
+                        if (tid == 0) {
+                            sel.thr_bins = bins;
+                            sel.thr_bstar = bstar;
+                            sel.thr_valid = 1;
+                            mbar_arrive(m.thr());  // releases these writes to the waiting warp
+                        }
+                    };
+                    SelectSmem<kSelThreads>& ssm_g = *reinterpret_cast<SelectSmem<kSelThreads>*>(m.merge);
+                    select_row<kSelThreads>(keys, g.NB, p.kmax, list, ssm_g, head, threshold, SelectGroupSync());
+                    if (tid == 0 && !sel.thr_valid) mbar_arrive(m.thr());  // no threshold pass: nothing early
+                }
             } else {
                 select_row<kThreads>(keys, g.NB, p.kmax, list, ssm, head);
             }
@@ -1602,6 +1634,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         sel.count = 0;
         sel.publish = -1;
         sel.early_count = 0;
+        sel.thr_valid = 0;
     }
     gate_phase<D, BLK, DG>(&tmK, &tmV, p, f, m, old_ctr);
     fence_proxy_async_smem();  // the gate's use of the ring precedes the decode's copies into it
@@ -1656,7 +1689,7 @@ Layout make_layout(int G, bool with_refresh) {
     const int merge_bytes = max(kConsumerWarps * G * D * 4 + 2 * kConsumerWarps * G * 4,  // warp states
                                 with_refresh ? kGateScratchBytes : 0);                   // or the gate's scratch
     const int info_bytes = (kInfoWords + kMaxStages * kStageInfoWords) * 4;
-    const int bar_bytes = (2 * kMaxStages + 3 + kMaxGateStages) * 8;
+    const int bar_bytes = (2 * kMaxStages + 4 + kMaxGateStages) * 8;
     const int refresh_bytes = with_refresh ? (int)sizeof(PoolSmem<D>) + 16 : 0;
     const int sel_bytes = with_refresh ? (int)sizeof(SelList) : 0;
     const int tail = merge_bytes + info_bytes + bar_bytes + refresh_bytes + sel_bytes + 64;

@@ -276,7 +276,10 @@ def test_workspace_regions_are_disjoint_aligned_and_hold_every_index():
 
 def struct_sizes(D, G):
     pool = (POOL_THREADS // (D // 8)) * D * 4 + D * 4
-    sel_list = 4 * 3 + 4 * MAX_SEL_ROWS * 3 + 4 * MAX_SEL_ROWS * SELECT_HEAD  # count, publish, own_len; row, nsel, len; head
+    # count, publish, own_len, early_count; early_ids[MAX_STAGES]; thr_valid, thr_bstar; the threshold
+    # bins (20 bytes); row, nsel, len; head (the kernel asserts the same size)
+    sel_list = 4 * 4 + 4 * MAX_STAGES + 4 * 2 + 20 + 4 * MAX_SEL_ROWS * 3 + 4 * MAX_SEL_ROWS * SELECT_HEAD
+    assert sel_list == 4556
     return pool, sel_list
 
 
@@ -285,7 +288,7 @@ def make_layout(D, blk, G, with_refresh):
     stage = (2 * tile + G * D * 2 + 1023) // 1024 * 1024
     merge = max(CONSUMER_WARPS * G * D * 4 + 2 * CONSUMER_WARPS * G * 4, GATE_SCRATCH if with_refresh else 0)
     info = (INFO_WORDS + MAX_STAGES * STAGE_INFO_WORDS) * 4
-    bars = (2 * MAX_STAGES + 3 + MAX_GATE_STAGES) * 8  # full/empty, consumers, gate stages, helpers, W_q
+    bars = (2 * MAX_STAGES + 4 + MAX_GATE_STAGES) * 8  # full/empty, consumers, gate stages, helpers, W_q, threshold
     pool, sel_list = struct_sizes(D, G)
     refresh = pool + 16 if with_refresh else 0
     sel = sel_list if with_refresh else 0
