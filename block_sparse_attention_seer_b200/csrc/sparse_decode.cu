@@ -673,6 +673,7 @@ __device__ __forceinline__ void count_taken_row(unsigned int* tally, uint32_t ep
 
 // One row of the rows a CTA meets in its gate range.
 struct GateRow {
+    int gi;                    // gate index: the row's place in the gate's position order
     int r, b, kvh, L, NB, js;  // js: first block whose pooled key is refreshed
     int s0, s1;                // cached positions [s0, s1) this CTA scores
     int scored;                // the row's choice needs scores
@@ -732,6 +733,15 @@ using GateScratchSmallest = GateScratch<64, 64>;
 static_assert(offsetof(GateScratchSmallest, rows) >= sizeof(SelectSmem<kStepThreads>),
               "the selection's scratch before the gate rows");
 
+// The gate's row order. Rows fit the grid: row i. Rows outnumber the CTAs:
+// head-major (i = kvh * B + b), so the few consecutive rows a CTA gates share
+// one head's W_q, which then arrives by one bulk copy.
+__device__ __forceinline__ int gate_row(const StepParams& f, int Hkv, int i) {
+    if (f.gate_cpr > 0) return i;
+    const int B = f.rows / Hkv;
+    return (i % B) * Hkv + i / B;
+}
+
 // The gate. The R x NBmax pooled-key positions (row-major, the layout of
 // kpool) are cut into gate_ctas equal contiguous ranges (with rows <= SMs,
 // each row into the same whole number of ranges). Each CTA projects the
@@ -744,7 +754,7 @@ static_assert(offsetof(GateScratchSmallest, rows) >= sizeof(SelectSmem<kStepThre
 // decode; only blocks that compete (a refresh point before the last block)
 // are refreshed here. `old_ctr` (the launch counter before this CTA's add) is
 // valid in thread 0.
-template <int D, int BLK, int DG>
+template <int D, int BLK, int DG, bool kManyRows>
 __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const Params& p, const StepParams& f,
                            const Smem& m, unsigned long long old_ctr) {
     constexpr int kThreads = kStepThreads;
@@ -763,27 +773,44 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
     const long long h0 = (long long)blockIdx.x * V1 / G1;
     const long long h1 = (long long)(blockIdx.x + 1) * V1 / G1;
     const bool whole_rows = G1 == f.rows;  // one CTA per row: keys stay in shared memory
-    // Rows r with r * NBmax < h1, from the row holding h0: exactly the rows
-    // whose [first, last] covering-CTA interval contains this CTA (an empty
+    // Gate indices i with i * NBmax < h1, from the one holding h0: exactly the
+    // rows whose [first, last] covering-CTA interval contains this CTA (an empty
     // range strictly inside a row still counts for that row).
     const int r_stop = (int)((h1 + f.NBmax - 1) / f.NBmax);
     int chunk_it = 0;  // bulk copies consumed so far (the same count on every thread)
-    // Rows fit the grid (one row per CTA): W_q of the row's head arrives by one
-    // bulk copy into the last wq_stages gate stages, so no register loads sit
-    // in front of the length load and the first pooled-key copies; those
-    // stages join the ring once the projection has read them.
+    // When the first batch's rows share one head (always with one row per CTA), W_q of
+    // that head arrives by one bulk copy into the last wq_stages gate stages, so
+    // no register loads sit in front of the lengths and the first pooled-key
+    // copies; those stages join the ring once the projection has read them.
     const int wq_stages = f.wq_stages;
     const int n_first = f.n_gate_stages - wq_stages;  // gate stages free before the projection
     const float* wq_s = reinterpret_cast<const float*>(m.base + f.chunk_off + n_first * kGateChunkBytes);
-    if (wq_stages > 0 && tid == 0) {
-        const uint32_t bytes = (uint32_t)(DG * D * 4);
-        mbar_arrive_expect_tx(m.wq(), bytes);
-        bulk_load(m.sbase + (uint32_t)(f.chunk_off + n_first * kGateChunkBytes),
-                  f.w_q + (size_t)((int)(h0 / f.NBmax) % p.Hkv) * DG * D, bytes, m.wq());
+    int wq_uses = 0;  // W_q copies waited on so far: the phase of its barrier
+    auto order = [&](int i) { return kManyRows ? gate_row(f, p.Hkv, i) : i; };
+    if constexpr (!kManyRows) {
+        if (wq_stages > 0 && tid == 0) {
+            const uint32_t bytes = (uint32_t)(DG * D * 4);
+            mbar_arrive_expect_tx(m.wq(), bytes);
+            bulk_load(m.sbase + (uint32_t)(f.chunk_off + n_first * kGateChunkBytes),
+                      f.w_q + (size_t)((int)(h0 / f.NBmax) % p.Hkv) * DG * D, bytes, m.wq());
+        }
     }
 
-    for (int r = (int)(h0 / f.NBmax); r < r_stop;) {
-        const int nb = min(kMaxBatchRows, r_stop - r);
+    for (int gi0 = (int)(h0 / f.NBmax); gi0 < r_stop;) {
+        const int nb = min(kMaxBatchRows, r_stop - gi0);
+        const int kvh0 = order(gi0) % p.Hkv;
+        bool one_head = true;
+        if constexpr (kManyRows)
+            for (int k = 1; k < nb; ++k) one_head &= order(gi0 + k) % p.Hkv == kvh0;
+        // (first batch only: a later one starts its copies at the ring position the last
+        // batch left, which need not leave the W_q stages free)
+        const bool wq_on = wq_stages > 0 && (!kManyRows || (one_head && chunk_it == 0));
+        if (kManyRows && wq_on && tid == 0) {  // the first batch: its stages are untouched
+            const uint32_t bytes = (uint32_t)(DG * D * 4);
+            mbar_arrive_expect_tx(m.wq(), bytes);
+            bulk_load(m.sbase + (uint32_t)(f.chunk_off + n_first * kGateChunkBytes),
+                      f.w_q + (size_t)kvh0 * DG * D, bytes, m.wq());
+        }
         // ---- (1) before anything else reaches DRAM: the projection weights of the
         //      batch rows (first kQBatch outputs per warp), their lengths and
         //      group-mean queries -- all independent loads, issued together.
@@ -793,31 +820,32 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
         const int total_q = (h1 > h0 ? nb : 0) * DG;  // outputs ordered by batch row, then e
         int len_raw = 0, upd_raw = -1;
         if (tid < nb) {
-            const int b = (r + tid) / p.Hkv;
+            const int b = order(gi0 + tid) / p.Hkv;
             len_raw = load_early(p.seq_lens + b);
             if (f.upd_start) upd_raw = load_early(f.upd_start + b);
         }
         WVec w[kQBatch];
-        if (total_q > 0 && wq_stages == 0) {
+        if (total_q > 0 && !wq_on) {
 #pragma unroll
             for (int u = 0; u < kQBatch; ++u) {
                 const int o = min(warp + u * kWarps, total_q - 1);
                 const int k = o / DG, e = o % DG;
-                const int kvh = (r + k) % p.Hkv;
+                const int kvh = order(gi0 + k) % p.Hkv;
                 load_early(w[u], f.w_q + ((size_t)kvh * DG + e) * D + lane * kVecD);
             }
         }
 
         if (tid < nb) {
             GateRow& g = sm.rows[tid];
-            g.r = r + tid;
+            g.gi = gi0 + tid;
+            g.r = order(g.gi);
             g.b = g.r / p.Hkv;
             g.kvh = g.r - g.b * p.Hkv;
             g.L = clamp_len(len_raw, p.Lmax);
             g.NB = (g.L + BLK - 1) / BLK;
             const int st0 = max(f.upd_start ? upd_raw : g.L - 1, 0);  // as refresh_start_block
             g.js = g.NB > 0 ? min(st0 / BLK, g.NB) : g.NB;
-            const long long rs = (long long)g.r * f.NBmax;
+            const long long rs = (long long)g.gi * f.NBmax;
             const int i0 = (int)(h0 > rs ? h0 - rs : 0);
             const int i1 = (int)((h1 - rs) < f.NBmax ? (h1 - rs) : f.NBmax);
             const int kb = p.kmax < g.NB ? p.kmax : g.NB;
@@ -856,40 +884,53 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
         // ---- (2) stream the cached pooled keys; meanwhile project the batch rows' queries.
         //      One row per CTA: thread 0 wrote the row itself and issues its first
         //      copies before the group-mean query.
-        if (tid == 0 && wq_stages > 0) {  // nb == 1: the row thread 0 just wrote
+        if (tid == 0 && wq_on && nb == 1) {  // the row thread 0 just wrote
             const int n0 = count_chunks();
             for (int i = 0; i < min(n_first, n0); ++i) issue(i);
         }
         if (total_q > 0) {
-            // one row per CTA: warp 0 stays free for the length and the copies
-            const int q0 = wq_stages > 0 ? 32 : 0;
+            // W_q by bulk copy: warp 0 stays free for the lengths and the copies
+            const int q0 = wq_on ? 32 : 0;
             for (int idx = tid - q0; idx >= 0 && idx < nb * D; idx += kThreads - q0) {
                 const int k = idx / D, d = idx - k * D;
-                const int row = r + k, b = row / p.Hkv, kvh = row - b * p.Hkv;
+                const int row = order(gi0 + k), b = row / p.Hkv, kvh = row - b * p.Hkv;
                 sm.qbar[k][d] = group_query_mean_at(p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G) * D, p.G, D, d);
             }
         }
         __syncthreads();
         const int total_chunks = count_chunks();
-        if (tid == 0 && wq_stages == 0)
-            for (int i = 0; i < min(f.n_gate_stages, total_chunks); ++i) issue(i);
-        if (wq_stages > 0) {
-            // the same pieces and sums as the register path below (equal bits)
+        if (tid == 0 && !(wq_on && nb == 1))
+            for (int c = 0; c < min(wq_on ? n_first : f.n_gate_stages, total_chunks); ++c) issue(c);
+        if (wq_on) {
+            // the same pieces and sums as the register path below (equal bits); one
+            // W_q row piece serves every row of the batch
             constexpr int kPerWarp = (DG + kWarps - 1) / kWarps;
-            if (!mbar_wait(m.wq(), 0u)) record_failure(m.info);
+            if (!mbar_wait(m.wq(), (uint32_t)(wq_uses & 1))) record_failure(m.info);
+            ++wq_uses;
 #pragma unroll 1
-            for (int u0 = 0; u0 < kPerWarp; u0 += 4) {  // four outputs per warp in flight
+            for (int u0 = 0; u0 < kPerWarp; u0 += 4) {  // four W_q rows per warp in flight
                 WVec wv[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int e = min(warp + (u0 + u) * kWarps, DG - 1);
                     wv[u] = *reinterpret_cast<const WVec*>(wq_s + (size_t)e * D + lane * kVecD);
                 }
+                if (!kManyRows || nb == 1) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = warp + (u0 + u) * kWarps;
-                    const float x = warp_sum(piece_dot(wv[u], &sm.qbar[0][lane * kVecD]));
-                    if (lane == 0 && e < DG) sm.qg[0][e] = x;
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = warp + (u0 + u) * kWarps;
+                        const float x = warp_sum(piece_dot(wv[u], &sm.qbar[0][lane * kVecD]));
+                        if (lane == 0 && e < DG) sm.qg[0][e] = x;
+                    }
+                } else {
+#pragma unroll 1
+                    for (int k = 0; k < nb; ++k)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = warp + (u0 + u) * kWarps;
+                            const float x = warp_sum(piece_dot(wv[u], &sm.qbar[k][lane * kVecD]));
+                            if (lane == 0 && e < DG) sm.qg[k][e] = x;
+                        }
                 }
             }
             fence_proxy_async_smem();  // these generic reads of W_q precede the copies into its stages
@@ -921,8 +962,8 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
             }
         }
         __syncthreads();
-        if (tid == 0 && wq_stages > 0)  // the W_q stages are read: they join the ring
-            for (int i = n_first; i < min(f.n_gate_stages, total_chunks); ++i) issue(i);
+        if (tid == 0 && wq_on)  // the W_q stages are read: they join the ring
+            for (int c = n_first; c < min(f.n_gate_stages, total_chunks); ++c) issue(c);
 
         // ---- (3) refresh and score competing blocks of a refresh point inside the range (multi-token appends)
         for (int k = 0; k < nb; ++k) {
@@ -975,7 +1016,7 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
         __syncthreads();  // every key of the batch written before the adds
         if (tid < nb) {
             const GateRow& g = sm.rows[tid];
-            const long long rs = (long long)g.r * f.NBmax;
+            const long long rs = (long long)g.gi * f.NBmax;
             if (whole_rows) {
                 sm.last_of[tid] = 1;  // the only CTA of its row
             } else {
@@ -1106,7 +1147,7 @@ __device__ void gate_phase(const CUtensorMap* tmK, const CUtensorMap* tmV, const
         }
         fence_proxy_async_smem();
         __syncthreads();  // scratch, keys and stages are reused by the next batch
-        r += nb;
+        gi0 += nb;
     }
 }
 
@@ -1345,7 +1386,8 @@ __device__ void step_producer(const CUtensorMap* tmK, const CUtensorMap* tmV, co
     int home_lo, home_hi;
     home_lo = (int)((long long)blockIdx.x * R / gridDim.x);
     home_hi = (int)((long long)(blockIdx.x + 1) * R / gridDim.x);
-    for (int row = home_lo; ok && row < home_hi; ++row) {
+    for (int hr = home_lo; ok && hr < home_hi; ++hr) {
+        const int row = gate_row(f, p.Hkv, hr);
         bool mine = false;
         for (int i = 0; i < nselrows; ++i) mine |= sel.row[i] == row;
         if (mine) continue;
@@ -1596,12 +1638,13 @@ __device__ void step_helpers(const Params& p, const StepParams& f, const Smem& m
     auto hsync = [&]() {
         if (ok) ok = warp_group_sync(m.helper(), hph, m.info);
     };
-    for (int r = (int)(h0 / f.NBmax); ok && (long long)r * f.NBmax < h1; ++r) {
+    for (int gi = (int)(h0 / f.NBmax); ok && (long long)gi * f.NBmax < h1; ++gi) {
+        const int r = gate_row(f, p.Hkv, gi);
         const int b = r / p.Hkv, kvh = r - b * p.Hkv;
         const int L = clamp_len(p.seq_lens[b], p.Lmax);
         const int NB = (L + BLK - 1) / BLK;
         if (NB == 0) continue;
-        const long long last = (long long)r * f.NBmax + NB - 1;
+        const long long last = (long long)gi * f.NBmax + NB - 1;
         if (last < h0 || last >= h1) continue;
         if (refresh_start_block(f, b, L, NB, BLK) > NB - 1) continue;
         const int j = NB - 1;
@@ -1617,7 +1660,9 @@ __device__ void step_helpers(const Params& p, const StepParams& f, const Smem& m
     }
 }
 
-template <int D, int BLK, int DG>
+// kManyRows: rows outnumber the CTAs (the gate takes batches of rows, head-major);
+// else one row per CTA. Two kernels, so neither mode's code shapes the other's.
+template <int D, int BLK, int DG, bool kManyRows>
 __global__ void __launch_bounds__(kStepThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const Params p, const StepParams f) {
@@ -1636,7 +1681,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         sel.early_count = 0;
         sel.thr_valid = 0;
     }
-    gate_phase<D, BLK, DG>(&tmK, &tmV, p, f, m, old_ctr);
+    gate_phase<D, BLK, DG, kManyRows>(&tmK, &tmV, p, f, m, old_ctr);
     fence_proxy_async_smem();  // the gate's use of the ring precedes the decode's copies into it
     if (threadIdx.x == 0) {
         const uint32_t epoch = epoch_of(old_ctr);
@@ -1800,7 +1845,9 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     const int n_gate = (ring - keys_bytes) / kGateChunkBytes;
     if (n_gate < 1) return cudaErrorInvalidConfiguration;
     static bool attr_done[kMaxSmemDevices] = {};
-    cudaError_t e = allow_big_smem(decode_step_kernel<D, BLK, DG>, attr_done);
+    static bool attr_done_many[kMaxSmemDevices] = {};
+    cudaError_t e = allow_big_smem(decode_step_kernel<D, BLK, DG, false>, attr_done);
+    if (e == cudaSuccess) e = allow_big_smem(decode_step_kernel<D, BLK, DG, true>, attr_done_many);
     if (e != cudaSuccess) return e;
     const int kmax = a.budget_tokens / s.blk;
     const StepGeometry geo = step_geometry(s, kmax, num_sms);
@@ -1848,9 +1895,10 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     // one CTA per row: decode stages that fit before the keys may start during the selection
     const int n_early = f.keys_off / l.stage_bytes < l.nst - 1 ? f.keys_off / l.stage_bytes : l.nst - 1;
     f.n_early = geo.gate_cpr == 1 ? n_early : 0;
-    // rows fit the grid: W_q of the row's head (dg x D fp32) first fills the last gate stages
+    // W_q of a batch's head (dg x D fp32; one row per CTA, or rows outnumbering the CTAs
+    // taken head-major) first fills the last gate stages
     const int wq_st = (DG * D * 4 + kGateChunkBytes - 1) / kGateChunkBytes;
-    f.wq_stages = (geo.gate_cpr > 0 && f.n_gate_stages > wq_st) ? wq_st : 0;
+    f.wq_stages = f.n_gate_stages > wq_st ? wq_st : 0;
 
     // One CTA per SM, all co-resident (the decode phase waits on rows that other CTAs publish).
     cudaLaunchConfig_t cfg = {};
@@ -1863,7 +1911,8 @@ cudaError_t step_impl(const Shape& s, const StepLaunch& a, const CUtensorMap& tm
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<D, BLK, DG>, tmK, tmV, p, f);
+    e = geo.gate_cpr > 0 ? cudaLaunchKernelEx(&cfg, decode_step_kernel<D, BLK, DG, false>, tmK, tmV, p, f)
+                         : cudaLaunchKernelEx(&cfg, decode_step_kernel<D, BLK, DG, true>, tmK, tmV, p, f);
     if (e != cudaSuccess) (void)cudaGetLastError();  // a rejected launch must not leak into the next call
     return e;
 }

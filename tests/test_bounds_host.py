@@ -96,6 +96,39 @@ def test_gate_ranges_cover_positions_once_and_counts_match(seed):
             assert count[r] == cl - cf + 1  # the kernel's count target for "last CTA of the row"
 
 
+def gate_row(i, B, Hkv, gate_cpr):
+    """The gate's row order: row i when rows fit the grid, else head-major (i = kvh * B + b)."""
+    return i if gate_cpr > 0 else (i % B) * Hkv + i // B
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_gate_order_is_a_permutation_and_ctas_mostly_share_one_head(seed):
+    """With more rows than CTAs, the gate visits rows head-major: every row once, its gate
+    index giving the positions [i * NBmax, (i + 1) * NBmax) the count target uses, and the
+    batches of consecutive indices a CTA gates mostly one head (one W_q bulk copy)."""
+    rng = random.Random(seed)
+    for _ in range(100):
+        Hkv = rng.choice([1, 2, 4, 8])
+        B = rng.randint(1, 300)
+        rows = B * Hkv
+        order = [gate_row(i, B, Hkv, 0) for i in range(rows)]
+        assert sorted(order) == list(range(rows))
+        assert [gate_row(i, B, Hkv, 1) for i in range(rows)] == list(range(rows))
+        NBmax, G1 = rng.randint(1, 600), 148
+        if rows <= G1:
+            continue
+        V1 = rows * NBmax
+        mixed = 0
+        for c in range(G1):
+            h0, h1 = c * V1 // G1, (c + 1) * V1 // G1
+            first, stop = h0 // NBmax, (h1 + NBmax - 1) // NBmax
+            for b0 in range(first, stop, 8):  # batches of up to 8 rows
+                heads = {gate_row(i, B, Hkv, 0) % Hkv for i in range(b0, min(stop, b0 + 8))}
+                mixed += len(heads) > 1
+        # a batch spans two heads only where the CTA's range crosses a head boundary
+        assert mixed <= Hkv - 1 + G1 * max(0, (8 * Hkv) // B), (B, Hkv, mixed)
+
+
 # ---------------------------------------------------------------- decode: fixed parts when rows fit
 
 @pytest.mark.parametrize("cpr", [1, 2, 3, 7, 18, 32, 148])
