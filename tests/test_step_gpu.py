@@ -81,8 +81,8 @@ def test_fused_tiny(seed):
     (2, 4, 2, 128, 64, 64, 3000, [2999, 1500], 640),
     (5, 8, 2, 128, 128, 64, 512, [0, 1, 64, 512, 300], 64),
     (5, 8, 2, 128, 128, 64, 512, [0, 1, 64, 512, 300], 4096),
-    # 2 rows of 1024 blocks: 32 gate CTAs per row, but only 8 kept blocks -> 8 one-block parts, 8 slots
-    (1, 8, 2, 128, 128, 64, 65536, [65536, 40001], 512),
+    # 4 rows of up to 1024 blocks: 32 gate CTAs per row, but only 8 kept blocks -> 8 one-block parts, 8 slots
+    (2, 8, 2, 128, 128, 64, 65536, [65536, 40001], 512),
 ])
 def test_fused_small_shapes(shape):
     B, Hq, Hkv, D, dg, blk, Lmax, lens, budget = shape
@@ -147,6 +147,29 @@ def test_fused_launch_epochs_rows_fit_the_grid():
     assert int(ws[:8].view(torch.int64).item()) == 3 * sms
     assert np.all(state[:, 0] == 3)  # published by the third call
     assert np.all(state[:, 4] == 0)  # one CTA per row: no partial slot was counted
+    assert api.seer_decode_wait_failures() == 0
+
+
+@pytest.mark.parametrize("case", ["tied_keys", "keep_all"])
+def test_fused_one_row_per_cta_selection_without_threshold_pass(case):
+    # 80 rows, one CTA each: the last warp waits for the selection's first threshold bin
+    # to start the decode early. With every pooled key of a row equal (a constant K
+    # along the sequence) the selection has no histogram pass (one key value: the
+    # lowest indices), and with a budget above every row's length it keeps all
+    # blocks without searching; either way the waiting warp must be released after
+    # the selection, with nothing issued early.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B = sms // 16 + 1  # x 8 heads: more than half the SMs, so one CTA per row
+    Lmax = 2048
+    budget = 512 if case == "tied_keys" else Lmax
+    wl = W.Workload("noearly", B, 32, 8, 128, 128, 64, Lmax, budget)
+    lens = np.array([Lmax - 50 * b for b in range(B)], np.int32)
+    inp = W.make_inputs(wl, seed=23, seq_lens=lens)
+    if case == "tied_keys":
+        inp["k_cache"][:] = inp["k_cache"][:, :, :1, :]
+    fus, _, _, _ = check_step(wl, to_dev(inp))
+    if case == "keep_all":
+        assert np.all(fus.num_selected.cpu().numpy() == (lens[:, None] + 63) // 64)
     assert api.seer_decode_wait_failures() == 0
 
 
