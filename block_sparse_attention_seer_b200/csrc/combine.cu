@@ -21,6 +21,7 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, int S, int BH,
                    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+    after_prior_grid();
     constexpr int kVec = D / 32;
     const int lane = threadIdx.x & 31;
     const int bh = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
@@ -87,10 +88,10 @@ cudaError_t launch_combine(const Shape& s, const float* o_part, const float* lse
     const int grid = (BH + kWarpsPerCta - 1) / kWarpsPerCta;
     auto* o = static_cast<__nv_bfloat16*>(out);
     if (s.D == 128)
-        combine_kernel<128><<<grid, kWarpsPerCta * 32, 0, stream>>>(o_part, lse_part, num_splits, BH, o, lse_out);
-    else
-        combine_kernel<64><<<grid, kWarpsPerCta * 32, 0, stream>>>(o_part, lse_part, num_splits, BH, o, lse_out);
-    return cudaGetLastError();
+        return launch_after_prior(combine_kernel<128>, dim3(grid), dim3(kWarpsPerCta * 32), 0, stream, nullptr,
+                                  o_part, lse_part, num_splits, BH, o, lse_out);
+    return launch_after_prior(combine_kernel<64>, dim3(grid), dim3(kWarpsPerCta * 32), 0, stream, nullptr, o_part,
+                              lse_part, num_splits, BH, o, lse_out);
 }
 
 }  // namespace seer

@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(kThreads)
     gate_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w_q,
                        const float* __restrict__ kpool, const int32_t* __restrict__ seq_lens,
                        float* __restrict__ scores, int Hq, int Hkv, int G, int blk, int Lmax, int NBmax) {
+    after_prior_grid();
     __shared__ float qbar[D];
     __shared__ float qg_part[DG];  // components this CTA projects (others stay unused)
     __shared__ __align__(16) float qg[DG];
@@ -82,20 +83,14 @@ __global__ void __launch_bounds__(kThreads)
 template <int D, int DG>
 cudaError_t launch_impl(const Shape& s, const void* q, const float* w_q, const float* kpool,
                         const int32_t* seq_lens, float* scores, int csize, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(csize, s.B * s.Hkv, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = csize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gate_scores_kernel<D, DG>, static_cast<const __nv_bfloat16*>(q), w_q, kpool,
-                              seq_lens, scores, s.Hq, s.Hkv, s.G, s.blk, s.Lmax, s.NBmax);
+    cudaLaunchAttribute cluster;
+    cluster.id = cudaLaunchAttributeClusterDimension;
+    cluster.val.clusterDim.x = csize;
+    cluster.val.clusterDim.y = 1;
+    cluster.val.clusterDim.z = 1;
+    return launch_after_prior(gate_scores_kernel<D, DG>, dim3(csize, s.B * s.Hkv, 1), dim3(kThreads, 1, 1), 0, stream,
+                              &cluster, static_cast<const __nv_bfloat16*>(q), w_q, kpool, seq_lens, scores, s.Hq,
+                              s.Hkv, s.G, s.blk, s.Lmax, s.NBmax);
 }
 
 }  // namespace

@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(kThreads)
     kpool_update_kernel(const __nv_bfloat16* __restrict__ k_cache, const float* __restrict__ w_k,
                         const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ upd_start,
                         float* __restrict__ kpool, int Hkv, int Lmax, int dg, int NBmax, int chunks) {
+    after_prior_grid();
     __shared__ PoolSmem<D> sm;
     const int row = blockIdx.y;
     const int b = row / Hkv, kvh = row - b * Hkv;
@@ -59,14 +60,15 @@ cudaError_t launch_kpool_update(const Shape& s, const void* k_cache, const float
     const dim3 grid(chunks, rows);
     const auto* k = static_cast<const __nv_bfloat16*>(k_cache);
 #define SEER_KPOOL(D_, B_)                                                                                       \
-    kpool_update_kernel<D_, B_><<<grid, kThreads, 0, stream>>>(k, w_k, seq_lens, upd_start, kpool, s.Hkv, s.Lmax, \
-                                                               s.dg, s.NBmax, chunks)
-    if (s.D == 128 && s.blk == 64) SEER_KPOOL(128, 64);
-    else if (s.D == 128) SEER_KPOOL(128, 128);
-    else if (s.blk == 64) SEER_KPOOL(64, 64);
-    else SEER_KPOOL(64, 128);
+    launch_after_prior(kpool_update_kernel<D_, B_>, grid, dim3(kThreads), 0, stream, nullptr, k, w_k, seq_lens,   \
+                       upd_start, kpool, s.Hkv, s.Lmax, s.dg, s.NBmax, chunks)
+    cudaError_t e;
+    if (s.D == 128 && s.blk == 64) e = SEER_KPOOL(128, 64);
+    else if (s.D == 128) e = SEER_KPOOL(128, 128);
+    else if (s.blk == 64) e = SEER_KPOOL(64, 64);
+    else e = SEER_KPOOL(64, 128);
 #undef SEER_KPOOL
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace seer

@@ -226,4 +226,31 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
 
 __device__ __forceinline__ int clamp_len(int len, int lmax) { return len < 0 ? 0 : (len > lmax ? lmax : len); }
 
+// Kernels of the separate calls are launched so that they may start while the
+// stream's previous kernel finishes (programmatic dependent launch). Each one
+// first waits for that kernel's completion and the visibility of its writes,
+// then lets the stream's next kernel launch: nothing is read early.
+__device__ __forceinline__ void after_prior_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Host side: launch `kernel` with that permission (and the given extra attribute, if any).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after_prior(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                               const cudaLaunchAttribute* extra, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (extra) attr[1] = *extra;
+    cfg.attrs = attr;
+    cfg.numAttrs = extra ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace seer

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(kThreads)
     select_blocks_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int Hkv, int Lmax,
                          int blk, int NBmax, int kmax, int32_t* __restrict__ block_idx,
                          int32_t* __restrict__ num_selected) {
+    after_prior_grid();
     extern __shared__ uint32_t keys[];  // [NBmax]
     __shared__ SelectSmem<kThreads> sm;
     const int row = blockIdx.x;
@@ -49,9 +50,8 @@ cudaError_t launch_select_blocks(const Shape& s, const float* scores, const int3
             attr_done = true;
         }
     }
-    select_blocks_kernel<<<rows, kThreads, smem, stream>>>(scores, seq_lens, s.Hkv, s.Lmax, s.blk, s.NBmax, kmax,
-                                                           block_idx, num_selected);
-    return cudaGetLastError();
+    return launch_after_prior(select_blocks_kernel, dim3(rows), dim3(kThreads), smem, stream, nullptr, scores,
+                              seq_lens, s.Hkv, s.Lmax, s.blk, s.NBmax, kmax, block_idx, num_selected);
 }
 
 }  // namespace seer

@@ -564,6 +564,7 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 1)  // 9 warps are allocated registers as 12: <= 168 each
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const Params p) {
+    after_prior_grid();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const Smem m = setup_smem(smem_raw, p);
     const long long g0 = (long long)blockIdx.x * p.V / p.P;
@@ -1797,8 +1798,8 @@ cudaError_t launch_impl(const Shape& s, const DecodeLaunch& a, const CUtensorMap
     cudaError_t e = allow_big_smem(sparse_decode_kernel<D, BLK>, attr_done);
     if (e != cudaSuccess) return e;
     const Params p = make_params<D, BLK>(s, a, l, sparse_decode_ctas(s, a.kmax, a.num_splits, num_sms));
-    sparse_decode_kernel<D, BLK><<<p.P, kThreads, l.total, stream>>>(tmK, tmV, p);
-    return cudaGetLastError();
+    return launch_after_prior(sparse_decode_kernel<D, BLK>, dim3(p.P), dim3(kThreads), l.total, stream, nullptr, tmK,
+                              tmV, p);
 }
 
 // How the fused step spreads its work (the same on the host and in the workspace layout).
